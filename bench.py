@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 BitStack residual-block linear (bs_linear).
+
+Headline (default): one decode call y = x W_hat^T of a 4096 x 4096 linear with n = 8
+loaded residual blocks, k = 16, batch 1, fp16 x -- microseconds per call and the
+fraction of the HBM / tensor roofline.  A step is one bs_linear call; steps rotate
+over enough distinct stacks (each with its own x and y) that the bytes touched
+between two uses of one stack exceed three times the L2 size.  Steps are replayed
+from CUDA graphs and timed with CUDA events on the launching stream; nvidia-smi
+clocks are sampled during the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same workload on its
+own GPU (the path needs no exchange between GPUs: replicas); the time is the max over
+ranks and the value is that time divided by all calls of all ranks.
+
+--impl reference times the CPU oracle (float64 NumPy) on the same workload, on a
+bounded sample, on the host cores.  The blocks are synthetic (random signs and
+factors of decomposition-like scale): timing depends only on shapes and bytes.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "bs_linear µs/call & % roofline (HBM/tensor) at 4096², n=8, k=16, batch 1"
+UNIT = "us/call"
+M_HEAD, D_HEAD, N_HEAD, K_HEAD, B_HEAD = 4096, 4096, 8, 16, 1
+L2_FALLBACK = 126 * 2 ** 20
+
+
+# ------------------------------------------------------------------ helpers -------
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def algorithmic(m, d, k, n, b):
+    """Bytes and FLOPs one call must move / do (the roofline's numerators)."""
+    block = m * d // 8 + 2 * k * (m + d)
+    nbytes = n * block + 2 * b * d + 2 * b * m + 4 * d
+    flops_factored = 2 * m * d * k * b * n      # the +-1 contraction S_i (x' (.) V_i)
+    flops_rebuild = 2 * m * d * (k * n + b)      # rank-k rebuild + dense product
+    return nbytes, flops_factored, flops_rebuild
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu_index), "-lms", "50"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kind):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = [os.path.join(ROOT, "residual_block_decomp_b200", "csrc", s) for s in rec["sources"]]
+        if rec["source_sha"] != source_sha(src):
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------- CUDA arm ---------
+def make_records(m, d, k, n, gen):
+    """n synthetic block records: random sign words (random bits in any bit order
+    are random bits) followed by fp16 U and V of decomposition-like scale."""
+    from residual_block_decomp_b200.layer import record_from_parts
+    recs = []
+    for i in range(n):
+        words = gen.integers(0, 2 ** 32, size=m * d // 32, dtype=np.uint64).astype(np.uint32)
+        U = wl.random_factors(m, k, gen, 0.12 / np.sqrt(i + 1.0))
+        V = wl.random_factors(d, k, gen, 0.12 / np.sqrt(i + 1.0))
+        recs.append(record_from_parts(words, U, V))
+    return recs
+
+
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    import residual_block_decomp_b200 as R
+    from residual_block_decomp_b200 import BitStackLinear
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    m, d, k, n, b = args.m, args.d, K_HEAD, args.n, args.batch
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 0) or L2_FALLBACK)
+    nbytes, flops_f, flops_r = algorithmic(m, d, k, n, b)
+    n_stacks = max(2, int(np.ceil(3 * l2 / nbytes)) + 1)
+
+    gen = wl.generator(2, 100 + rank, "blocks")
+    inv_s = wl.synthetic_inv_scale(d, gen)
+    layers, xs, ys = [], [], []
+    for j in range(n_stacks):
+        layer = BitStackLinear(m, d, n, inv_s, device=dev)
+        for rec in make_records(m, d, k, n, gen):
+            layer.add_record(rec)
+        layer.set_loaded(n)
+        layers.append(layer)
+        xs.append(torch.from_numpy(wl.activations(b, d, gen).astype(np.float16)).to(dev))
+        ys.append(torch.empty((b, m), dtype=torch.float16, device=dev))
+    ws = torch.zeros(R.bs_workspace_bytes(m, d, k, n, b), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+
+    stream = torch.cuda.Stream(dev)
+
+    def step(j):
+        layers[j % n_stacks].forward(xs[j % n_stacks], n, out=ys[j % n_stacks], workspace=ws, stream=stream)
+
+    # warm-up (eager), then graphs of whole rotations
+    with torch.cuda.stream(stream):
+        for j in range(max(args.warmup, 3)):
+            step(j)
+    stream.synchronize()
+    per_graph = min(args.steps, n_stacks * max(1, 2000 // n_stacks))
+    reps, rem = divmod(args.steps, per_graph)
+
+    def capture(count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(count):
+                step(j)
+        return g
+
+    g_main = capture(per_graph)
+    g_rem = capture(rem) if rem else None
+    with torch.cuda.stream(stream):     # replay() launches on the current stream
+        g_main.replay()
+    stream.synchronize()
+    assert layers[0].device_error() == 0, "device error during warm-up"
+
+    def timed(run):
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]) as cs:
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                run()
+                e1.record(stream)
+            e1.synchronize()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1), cs.summary()
+
+    def run_main():
+        for _ in range(reps):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    ms, clocks = timed(run_main)
+    for layer in layers[:1]:
+        assert layer.device_error() == 0, "device error in the timed region"
+
+    # ------------------------------------------------------------------ e2e ----
+    # through the C ABI with host buffers: pinned x -> device, bs_linear, y -> pinned host
+    xh = [torch.empty((b, d), dtype=torch.float16, pin_memory=True) for _ in range(n_stacks)]
+    yh = [torch.empty((b, m), dtype=torch.float16, pin_memory=True) for _ in range(n_stacks)]
+    for j in range(n_stacks):
+        xh[j].copy_(xs[j].cpu())
+
+    def e2e_step(j):
+        jj = j % n_stacks
+        xs[jj].copy_(xh[jj], non_blocking=True)
+        step(jj)
+        yh[jj].copy_(ys[jj], non_blocking=True)
+
+    def capture_e2e(count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(count):
+                e2e_step(j)
+        return g
+
+    e2e_steps = args.e2e_steps or args.steps
+    per_e = min(e2e_steps, per_graph)
+    reps_e, rem_e = divmod(e2e_steps, per_e)
+    ge_main = capture_e2e(per_e)
+    ge_rem = capture_e2e(rem_e) if rem_e else None
+    with torch.cuda.stream(stream):
+        ge_main.replay()
+    stream.synchronize()
+
+    def run_e2e():
+        for _ in range(reps_e):
+            ge_main.replay()
+        if ge_rem is not None:
+            ge_rem.replay()
+
+    ms_e2e, _ = timed(run_e2e)
+
+    # max over ranks
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+
+    out = {
+        "ms": ms, "ms_e2e": ms_e2e, "steps": args.steps, "e2e_steps": e2e_steps, "clocks": clocks,
+        "n_stacks": n_stacks, "l2": l2, "bytes": nbytes, "flops_factored": flops_f, "flops_rebuild": flops_r,
+        "e2e_h2d": b * d * 2, "e2e_d2h": b * m * 2,
+    }
+    if args.extras and rank == 0:
+        out["extras"] = extras(args, dev, stream, layers[0], ws, inv_s)
+    for layer in layers:
+        layer.close()
+    return out
+
+
+def extras(args, dev, stream, layer, ws, inv_s):
+    """Secondary figures (not the headline): n sweep, batch 4, prefill, block load."""
+    import torch
+    res = {}
+    m, d, k = args.m, args.d, K_HEAD
+
+    def time_calls(fn, count=200):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(count):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / count
+
+    x1 = torch.randn((1, d), device=dev).half()
+    y1 = torch.empty((1, m), device=dev, dtype=torch.float16)
+    res["decode_b1_us_by_n"] = {
+        str(nn): round(time_calls(lambda nn=nn: layer.forward(x1, nn, out=y1, workspace=ws, stream=stream)), 3)
+        for nn in range(1, args.n + 1)}
+    x4 = torch.randn((4, d), device=dev).half()
+    y4 = torch.empty((4, m), device=dev, dtype=torch.float16)
+    ws4 = torch.zeros(layer.workspace(args.n, 4).numel(), dtype=torch.uint8, device=dev)
+    res["decode_b4_n8_us"] = round(time_calls(lambda: layer.forward(x4, args.n, out=y4, workspace=ws4,
+                                                                     stream=stream)), 3)
+    for M in (512, 4096):
+        xM = torch.randn((M, d), device=dev).bfloat16()
+        yM = torch.empty((M, m), device=dev, dtype=torch.bfloat16)
+        us = time_calls(lambda: layer.forward(xM, args.n, out=yM, stream=stream), count=20)
+        res[f"prefill_M{M}_us"] = round(us, 2)
+        res[f"prefill_M{M}_gemm_tflops"] = round(2.0 * M * m * d / (us * 1e-6) / 1e12, 1)
+    # block load: one record H2D (pinned host -> device) per append
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    layer.set_loaded(0)
+    torch.cuda.synchronize(dev)
+    t0.record(torch.cuda.current_stream(dev))
+    layer.set_loaded(args.n)
+    t1.record(torch.cuda.current_stream(dev))
+    t1.synchronize()
+    per_block = t0.elapsed_time(t1) * 1000.0 / args.n
+    res["append_us_per_block"] = round(per_block, 1)
+    res["append_gbs"] = round(layer.block_bytes / (per_block * 1e-6) / 1e9, 1)
+    return res
+
+
+# -------------------------------------------------------------- oracle arm --------
+def run_oracle(args, budget_s):
+    """Times the oracle's factored float64 linear on the headline workload."""
+    from oracle import linear
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
+    except Exception:
+        threads = None
+    cores = len(os.sched_getaffinity(0))
+    m, d, k, n, b = args.m, args.d, K_HEAD, args.n, args.batch
+    gen = wl.generator(2, 900, "blocks")
+    negs, Us, Vs = [], [], []
+    for i in range(n):
+        neg, U, V = wl.synthetic_block(m, d, k, gen, level=i)
+        negs.append(neg)
+        Us.append(U)
+        Vs.append(V)
+    inv_s = wl.synthetic_inv_scale(d, gen)
+    x = wl.activations(b, d, gen).astype(np.float16)
+    calls = 0
+    t0 = time.perf_counter()
+    while True:
+        linear.linear_factored(x, negs, Us, Vs, inv_s, n, m)
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": el * 1e6 / calls, "unit": UNIT, "cores": threads or cores, "kind": "oracle",
+            "sample": f"{calls} call(s) of the float64 factored oracle on the full {m}x{d}, n={n}, k={k}, "
+                      f"batch {b} workload ({el:.1f} s); host has {cores} cores"}
+
+
+# ---------------------------------------------------------------------- main ------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=0)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--m", type=int, default=M_HEAD)
+    ap.add_argument("--d", type=int, default=D_HEAD)
+    ap.add_argument("--n", type=int, default=N_HEAD)
+    ap.add_argument("--batch", type=int, default=B_HEAD)
+    ap.add_argument("--no-extras", dest="extras", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    workload = f"decode {args.m}x{args.d} n={args.n} k={K_HEAD} batch={args.batch} fp16"
+    config = {"workload": workload, "m": args.m, "d": args.d, "n_loaded": args.n, "k": K_HEAD,
+              "batch": args.batch, "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cpu = run_oracle(args, budget_s=args.cpu_seconds)
+        v = cpu["value"]
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": cpu, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_cuda(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    hbm, bf16, bf16_sus, src = peaks()
+    us_step = res["ms"] * 1000.0 / args.steps                 # per call on one GPU
+    value = res["ms"] * 1000.0 / (args.steps * world)          # whole job: all calls of all ranks
+    nbytes = res["bytes"]
+    achieved = nbytes / (us_step * 1e-6) / 1e9                 # GB/s of the decode kernel
+    i8_peak = bf16 * 2.0                                       # int8 dense = 2x bf16 (nominal ratio 4.5 / 2.25)
+    t_roof = max(nbytes / (hbm * 1e9), res["flops_factored"] / (bf16 * 1e12))
+    traffic = dram_traffic("decode")
+    cpu = run_oracle(args, budget_s=args.cpu_seconds) if args.cpu_seconds > 0 else None
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us_step / 1000.0, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": dict(config, l2_policy=f"inputs larger than L2: {res['n_stacks']} distinct stacks "
+                                         f"({res['n_stacks'] * nbytes / 2**20:.0f} MiB) rotated, L2 "
+                                         f"{res['l2'] / 2**20:.0f} MiB", timing="CUDA graph replays, CUDA events"),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic, "peak_source": src,
+                     "t_roof_us": round(t_roof * 1e6, 3), "frac_of_roofline_time": round(t_roof * 1e6 / us_step, 4),
+                     "bytes_per_launch": nbytes,
+                     "tensor_i8_frac": round(2 * res["flops_factored"] * 1.0 / (us_step * 1e-6) / (i8_peak * 1e12), 4)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(res["ms_e2e"] * 1000.0 / (res["e2e_steps"] * world), 4), "unit": UNIT,
+                "h2d_bytes_per_step": res["e2e_h2d"], "d2h_bytes_per_step": res["e2e_d2h"]},
+        "gpu_launches": args.steps,
+        "clocks": res["clocks"],
+        "tokens_per_s": round(args.batch * 1e6 / value, 1),
+        "weights_per_s": round(args.m * args.d * 1e6 / value, 1),
+    }
+    if "extras" in res:
+        line["extras"] = res["extras"]
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

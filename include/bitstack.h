@@ -1,0 +1,190 @@
+/*
+ * bitstack.h -- C ABI of the B200 BitStack residual-block linear.
+ *
+ * What it computes.  A weight W (m x d, m = out_features, d = in_features) is held
+ * as a stack of residual blocks.  Block i is a sign matrix S_i in {+1,-1}^{m x d},
+ * packed one bit per entry, plus rank-k fp16 factors U_i (m x k) and V_i (d x k)
+ * with sqrt(sigma) folded into both.  The weight the first n blocks describe is
+ *
+ *     W_hat_n = ( sum_{i < n} S_i (.) (U_i V_i^T) ) diag(1/s),
+ *
+ * where 1/s (length d, fp32) undoes the activation-aware per-input-channel scaling
+ * applied before the decomposition.  bs_linear evaluates y = x W_hat_n^T for a
+ * batch of rows x straight from the packed stack: the dense weight is never written
+ * to device memory.
+ *
+ * Sources (page titles and the part of each page):
+ *  - residual block = packed sign matrix + singular vectors from absolute value
+ *    decomposition: "BitStack: Fine-Grained Size Control for Compressed Large
+ *    Language Models in Variable Memory Environments" (paper-review page), Fig. 3
+ *    caption; OpenReview discussion of "BitStack: Any-Size Compression of Large
+ *    Language Models in Variable Memory Environments", reply A1.A.
+ *  - W_hat as the sum of sign (.) (u_k vt_k) over the loaded blocks, starting from
+ *    a zero accumulator: same OpenReview discussion, weight restoration snippet.
+ *  - scaling undone per input channel: review page, Fig. 5 caption ("Eq. 4").
+ *  - blocks loaded from storage when memory grows and offloaded when it shrinks,
+ *    per weight, in a presorted order: review page, Fig. 2 caption; OpenReview
+ *    reply A1.B.
+ *
+ * Device record layout (one block, bs_block_bytes(m, d, k) bytes):
+ *   [ sign words : m*d/32 little-endian uint32, device tile order      ]
+ *   [ U          : m x k fp16, row-major                               ]
+ *   [ V          : d x k fp16, row-major                               ]
+ * Sign bit value 1 means S = -1.  Device tile order: the m x d sign matrix is cut
+ * into tiles of 128 rows x 256 columns stored row-tile-major (tile index
+ * rt * (d/256) + g); a tile is 1024 words (4 KiB).  Row rr of a tile owns 8 words
+ * p = 0..7 covering its 256 columns; word p of row rr is at index
+ * (p / 4) * 512 + rr * 4 + (p % 4) within the tile, and bit 8*q + t of that word
+ * (q = 0..3, t = 0..7) holds column 32*t + 4*p + q of the tile.  (This order lets a
+ * kernel turn the bits of one K-step of 32 columns into int8 operands with one
+ * shift-and-mask per 4 columns.)  bs_pack_record builds records from canonical
+ * bits on the host.
+ *
+ * Conventions for every call.
+ *  - Ownership: the caller allocates and owns all device memory (records, 1/s,
+ *    workspace, x, y, W_out) and all pinned host records; the library never calls
+ *    cudaMalloc or cudaFree.  A handle owns only its small host-side struct.
+ *  - Streams: bs_stream_t is a cudaStream_t (NULL = the legacy default stream).
+ *    Every device-side effect is ordered on the stream passed to the call.
+ *  - Errors: every call returns a bs_status.  Arguments are validated on the host
+ *    before anything is launched; a rejected call has no effect.  Launch failures
+ *    return BS_ERR_CUDA.  Device-side waits are bounded; a wait that runs out sets a
+ *    sticky device error word that bs_get_device_error reports as BS_ERR_TIMEOUT.
+ *  - Shapes: m % 128 == 0, d % 256 == 0, 128 <= m, d <= 65536, k == 16 on the GPU
+ *    path (bs_block_bytes and bs_pack_record accept any k >= 1).
+ *  - Alignment: device buffers 256-byte aligned; x, y, W_out and 1/s 16-byte
+ *    aligned.  Violations return BS_ERR_ALIGNMENT.
+ *  - Thread safety: a handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef BITSTACK_B200_H
+#define BITSTACK_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bs_stream_t; /* identical to cudaStream_t */
+typedef struct bs_stack_s* bs_stack_t;   /* opaque handle of one weight's block stack */
+
+typedef enum {
+  BS_OK = 0,
+  BS_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size, ... */
+  BS_ERR_UNSUPPORTED_SHAPE = 2, /* m, d, k outside the supported set */
+  BS_ERR_ALIGNMENT = 3,         /* a pointer misses its required alignment */
+  BS_ERR_CAPACITY = 4,          /* append beyond capacity, buffer too small */
+  BS_ERR_RANGE = 5,             /* n_loaded > blocks held, drop at zero, bad block index */
+  BS_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
+  BS_ERR_TIMEOUT = 7,           /* a bounded device-side wait ran out */
+  BS_ERR_NO_DEVICE = 8          /* no usable sm_100 device */
+} bs_status;
+
+typedef enum { BS_F16 = 0, BS_BF16 = 1, BS_F32 = 2 } bs_dtype;
+
+/* ------------------------------------------------------------------ sizes ------ */
+
+/* Bytes of one block record: m*d/8 + 2*k*(m + d).  This equals the fp16 size of a
+ * rank-k' plain-SVD block with k' = k + m*d/(16*(m + d)) (review page, Fig. 5
+ * caption), and gives 7,929,856 B = 7.56 MiB for 14336 x 4096 at k = 16, the
+ * largest block of an 8B model (OpenReview discussion, reply A1.A).
+ * Returns 0 for non-positive arguments or when d or m*d is not a multiple of 8. */
+size_t bs_block_bytes(int m, int d, int k);
+
+/* Device bytes the caller must provide for a stack of `capacity_blocks` blocks:
+ * capacity * bs_block_bytes (block i at offset i * bs_block_bytes) rounded up to
+ * 256, plus a small metadata area (per-block column maxima of |V_i| and the device
+ * error word).  0 on invalid arguments. */
+size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks);
+
+/* Workspace bytes bs_linear needs for `n_loaded` blocks and `batch` rows (0 when the
+ * call needs none).  The caller zeroes a workspace once before its first use (e.g.
+ * cudaMemsetAsync); the library keeps it consistent afterwards: its first 256 bytes
+ * hold a launch epoch that tags the flags and counters of each call, so no clearing
+ * is needed between calls, and calls captured in a CUDA graph may be replayed.  One
+ * workspace may serve any number of stacks whose calls are ordered on one stream;
+ * calls that may overlap on the GPU need distinct workspaces. */
+size_t bs_workspace_bytes(int m, int d, int k, int n_loaded, int batch);
+
+/* ---------------------------------------------------------- host packing ------ */
+
+/* Builds one block record on the host.
+ * neg_bits: m rows of d/8 bytes, canonical order (column c in bit c%8 of byte c/8,
+ *           1 = sign -1).  U: m x k fp16 bits, V: d x k fp16 bits, row-major.
+ * record:   bs_block_bytes(m, d, k) bytes written in the device layout above.
+ * Pure host code; needs no GPU.  m % 128 == 0 and d % 256 == 0 are required. */
+bs_status bs_pack_record(int m, int d, int k, const uint8_t* neg_bits, const uint16_t* U, const uint16_t* V,
+                         void* record);
+
+/* ------------------------------------------------------------ stack life ------ */
+
+/* Creates a handle over caller-owned device memory.
+ * dev_blocks: >= bs_stack_device_bytes(m, d, k, capacity_blocks) bytes, 256-aligned;
+ * dev_inv_scale: d fp32 values of 1/s, 16-aligned, read by every bs_linear call
+ * (kept by pointer: it must stay valid and unchanged while the handle is used).
+ * The stack starts with 0 blocks; the metadata area is cleared on `stream`.
+ * Fails with BS_ERR_NO_DEVICE when the current device is not sm_100. */
+bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                          const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out);
+
+/* Frees the host handle only; device memory stays with the caller. */
+bs_status bs_stack_destroy(bs_stack_t stack);
+
+/* Number of blocks currently held (loaded). */
+bs_status bs_stack_num_blocks(bs_stack_t stack, int* n_blocks);
+
+/* Loads the next block: one cudaMemcpyAsync of the record (ideally pinned host
+ * memory, which must stay valid until the stream passes the copy) into slot
+ * n_blocks, then a one-CTA kernel that stores max_c |V[c, j]| of the new block
+ * (used to pick the int8 scale of the decode kernel's activations).  n_blocks += 1.
+ * BS_ERR_CAPACITY when the stack is full. */
+bs_status bs_append_block(bs_stack_t stack, const void* host_record, bs_stream_t stream);
+
+/* Offloads the last block: n_blocks -= 1, no transfer (the host copy is the
+ * storage).  BS_ERR_RANGE when the stack is empty. */
+bs_status bs_drop_block(bs_stack_t stack);
+
+/* ----------------------------------------------------------------- compute ----- */
+
+/* y = x W_hat_n^T with n = n_loaded (0 <= n_loaded <= n_blocks).
+ * x: batch x d row-major, y: batch x m row-major, both of dtype `dt` (BS_F16 or
+ * BS_BF16), device pointers, 16-byte aligned.  n_loaded == 0 writes y = 0 (the
+ * restoration accumulator starts at zero).  batch <= 4 runs the decode kernel (the
+ * factored form y = sum_i U_i (S_i ((x (.) 1/s) V_i)) with the +-1 contraction on
+ * int8 tensor cores); larger batches run the prefill kernel (W_hat tiles rebuilt in
+ * shared memory, then a tcgen05 GEMM).  workspace: >= bs_workspace_bytes(m, d, k,
+ * n_loaded, batch) device bytes, 256-aligned, zeroed before its first use (may be
+ * NULL when the size is 0).  Asynchronous on `stream`; capturable in a CUDA graph. */
+bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
+                    void* workspace, size_t workspace_bytes, bs_stream_t stream);
+
+/* W_out = W_hat_n (m x d row-major, dtype BS_F32, BS_F16 or BS_BF16), for tests and
+ * for users who want the dense weight (the unfused path of the restoration
+ * snippet).  Asynchronous on `stream`. */
+bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_stream_t stream);
+
+/* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
+bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream);
+
+/* ------------------------------------------------------------------ errors ----- */
+
+/* Synchronises `stack`'s device, reads and clears the sticky device error word:
+ * BS_OK, BS_ERR_TIMEOUT (a bounded wait ran out), or BS_ERR_CUDA. */
+bs_status bs_get_device_error(bs_stack_t stack);
+
+/* Static text for a status code. */
+const char* bs_status_string(bs_status status);
+
+/* Sets the bound (nanoseconds) on every device-side wait of this stack's kernels
+ * (default 500 ms; values < 1000 are raised to 1000).  With `unreachable_flag`
+ * non-zero, the next bs_linear decode call waits for an activation-chunk flag
+ * that no CTA ever sets, so its waits run out: a host-side way to exercise the
+ * timeout path without faulting the GPU. */
+bs_status bs_debug_set_wait(bs_stack_t stack, long long timeout_ns, int unreachable_flag);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITSTACK_B200_H */

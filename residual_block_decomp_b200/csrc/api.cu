@@ -1,0 +1,322 @@
+// Host implementation of the C ABI declared in include/bitstack.h: argument checks,
+// the stack handle, block append/drop, host packing, and kernel dispatch.  The
+// library never allocates device memory; every device buffer comes from the caller.
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+using namespace bs;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool gpu_shape_ok(int m, int d, int k) {
+  return k == kK && m >= kTileRows && d >= kTileCols && m <= 65536 && d <= 65536 && m % kTileRows == 0 &&
+         d % kTileCols == 0;
+}
+
+size_t meta_bytes(int capacity) {
+  return align_up(static_cast<size_t>(capacity) * kK * sizeof(float) + 256, 256);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Tensor map over a tensor of fp16/bf16 elements; dims / strides innermost first,
+// strides in bytes for dims 1.., box in elements.  No swizzle, no interleave.
+bool encode(CUtensorMap* map, bool bf16, int rank, void* base, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<cuuint32_t>(rank),
+         base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool build_factor_maps(bs_stack_s* s) {
+  // U: dims {16 (j), m (rows), capacity (blocks)}, box {8, 128, 1}
+  // V: dims {16 (j), d (cols), capacity (blocks)}, box {8, 32, 1}
+  const cuuint64_t ustr[2] = {kK * 2, static_cast<cuuint64_t>(s->block_bytes)};
+  const cuuint64_t udims[3] = {kK, static_cast<cuuint64_t>(s->m), static_cast<cuuint64_t>(s->capacity)};
+  const cuuint32_t ubox[3] = {8, kTileRows, 1};
+  uint8_t* ubase = s->blocks + static_cast<size_t>(s->m) * s->d / 8;
+  const cuuint64_t vdims[3] = {kK, static_cast<cuuint64_t>(s->d), static_cast<cuuint64_t>(s->capacity)};
+  const cuuint32_t vbox[3] = {8, 32, 1};
+  uint8_t* vbase = ubase + static_cast<size_t>(2) * kK * s->m;
+  return encode(&s->tm_u, false, 3, ubase, udims, ustr, ubox) && encode(&s->tm_v, false, 3, vbase, vdims, ustr, vbox);
+}
+
+bs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BS_OK : BS_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t bs_block_bytes(int m, int d, int k) {
+  if (m <= 0 || d <= 0 || k <= 0 || d % 8 != 0) return 0;
+  return static_cast<size_t>(m) * d / 8 + static_cast<size_t>(2) * k * (static_cast<size_t>(m) + d);
+}
+
+size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks) {
+  if (!gpu_shape_ok(m, d, k) || capacity_blocks <= 0) return 0;
+  return align_up(static_cast<size_t>(capacity_blocks) * bs_block_bytes(m, d, k), 256) + meta_bytes(capacity_blocks);
+}
+
+size_t bs_workspace_bytes(int m, int d, int k, int n_loaded, int batch) {
+  if (!gpu_shape_ok(m, d, k) || n_loaded < 0 || batch <= 0) return 0;
+  if (n_loaded == 0 || batch > kDecodeMaxBatch) return 0;
+  return decode_ws_layout(m, d, n_loaded, batch).total;
+}
+
+bs_status bs_pack_record(int m, int d, int k, const uint8_t* neg_bits, const uint16_t* U, const uint16_t* V,
+                         void* record) {
+  if (neg_bits == nullptr || U == nullptr || V == nullptr || record == nullptr || k <= 0) return BS_ERR_INVALID_ARG;
+  if (m <= 0 || d <= 0 || m % kTileRows != 0 || d % kTileCols != 0) return BS_ERR_UNSUPPORTED_SHAPE;
+  uint8_t* out = static_cast<uint8_t*>(record);
+  const size_t row_bytes = static_cast<size_t>(d) / 8;
+  const int RT = m / kTileRows, KG = d / kTileCols;
+  for (int rt = 0; rt < RT; ++rt) {
+    for (int g = 0; g < KG; ++g) {
+      uint8_t* tile = out + (static_cast<size_t>(rt) * KG + g) * kTileBytes;
+      for (int rr = 0; rr < kTileRows; ++rr) {
+        const uint8_t* src = neg_bits + static_cast<size_t>(rt * kTileRows + rr) * row_bytes;
+        for (int pw = 0; pw < 8; ++pw) {
+          uint32_t word = 0;
+          for (int q = 0; q < 4; ++q) {
+            for (int t = 0; t < 8; ++t) {
+              const int c = g * kTileCols + 32 * t + 4 * pw + q;
+              const uint32_t bit = (src[c >> 3] >> (c & 7)) & 1u;
+              word |= bit << (8 * q + t);
+            }
+          }
+          const size_t widx = static_cast<size_t>(pw >> 2) * 512 + static_cast<size_t>(rr) * 4 + (pw & 3);
+          const uint8_t le[4] = {static_cast<uint8_t>(word), static_cast<uint8_t>(word >> 8),
+                                 static_cast<uint8_t>(word >> 16), static_cast<uint8_t>(word >> 24)};
+          std::memcpy(tile + widx * 4, le, 4);
+        }
+      }
+    }
+  }
+  const size_t nsb = static_cast<size_t>(m) * d / 8;
+  std::memcpy(out + nsb, U, static_cast<size_t>(m) * k * 2);
+  std::memcpy(out + nsb + static_cast<size_t>(m) * k * 2, V, static_cast<size_t>(d) * k * 2);
+  return BS_OK;
+}
+
+bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                          const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out) {
+  if (out == nullptr || dev_blocks == nullptr || dev_inv_scale == nullptr || capacity_blocks <= 0)
+    return BS_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!gpu_shape_ok(m, d, k)) return BS_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(dev_blocks, 256) || !aligned(dev_inv_scale, 16)) return BS_ERR_ALIGNMENT;
+  if (dev_bytes < bs_stack_device_bytes(m, d, k, capacity_blocks)) return BS_ERR_CAPACITY;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BS_ERR_NO_DEVICE;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return BS_ERR_NO_DEVICE;
+  if (major != 10 || minor != 0) return BS_ERR_NO_DEVICE;
+  bs_stack_s* s = new (std::nothrow) bs_stack_s();
+  if (s == nullptr) return BS_ERR_INVALID_ARG;
+  s->m = m;
+  s->d = d;
+  s->k = k;
+  s->capacity = capacity_blocks;
+  s->n_blocks = 0;
+  s->blocks = static_cast<uint8_t*>(dev_blocks);
+  s->block_bytes = bs_block_bytes(m, d, k);
+  s->dev_bytes = dev_bytes;
+  s->inv_s = dev_inv_scale;
+  s->vmax = reinterpret_cast<float*>(s->blocks + align_up(static_cast<size_t>(capacity_blocks) * s->block_bytes, 256));
+  s->err = reinterpret_cast<uint32_t*>(s->vmax + static_cast<size_t>(capacity_blocks) * kK);
+  s->device = dev;
+  s->sm_count = sms;
+  s->timeout_ns = 500000000ull;
+  s->inject_unreachable = 0;
+  s->tmaps_ready = build_factor_maps(s) ? 1 : 0;
+  const cudaError_t e = cudaMemsetAsync(s->vmax, 0, meta_bytes(capacity_blocks), stream);
+  if (e != cudaSuccess) {
+    delete s;
+    return BS_ERR_CUDA;
+  }
+  *out = s;
+  return BS_OK;
+}
+
+bs_status bs_stack_destroy(bs_stack_t stack) {
+  if (stack == nullptr) return BS_ERR_INVALID_ARG;
+  delete stack;
+  return BS_OK;
+}
+
+bs_status bs_stack_num_blocks(bs_stack_t stack, int* n_blocks) {
+  if (stack == nullptr || n_blocks == nullptr) return BS_ERR_INVALID_ARG;
+  *n_blocks = stack->n_blocks;
+  return BS_OK;
+}
+
+bs_status bs_append_block(bs_stack_t stack, const void* host_record, bs_stream_t stream) {
+  if (stack == nullptr || host_record == nullptr) return BS_ERR_INVALID_ARG;
+  if (stack->n_blocks >= stack->capacity) return BS_ERR_CAPACITY;
+  uint8_t* slot = stack->blocks + static_cast<size_t>(stack->n_blocks) * stack->block_bytes;
+  cudaError_t e = cudaMemcpyAsync(slot, host_record, stack->block_bytes, cudaMemcpyDefault, stream);
+  if (e != cudaSuccess) return BS_ERR_CUDA;
+  e = launch_vmax(slot, stack->m, stack->d, stack->vmax + static_cast<size_t>(stack->n_blocks) * kK, stream);
+  if (e != cudaSuccess) return BS_ERR_CUDA;
+  stack->n_blocks += 1;
+  return BS_OK;
+}
+
+bs_status bs_drop_block(bs_stack_t stack) {
+  if (stack == nullptr) return BS_ERR_INVALID_ARG;
+  if (stack->n_blocks <= 0) return BS_ERR_RANGE;
+  stack->n_blocks -= 1;
+  return BS_OK;
+}
+
+bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
+                    void* workspace, size_t workspace_bytes, bs_stream_t stream) {
+  if (stack == nullptr || x == nullptr || y == nullptr || batch <= 0) return BS_ERR_INVALID_ARG;
+  if (dt != BS_F16 && dt != BS_BF16) return BS_ERR_INVALID_ARG;
+  if (n_loaded < 0 || n_loaded > stack->n_blocks) return BS_ERR_RANGE;
+  if (!aligned(x, 16) || !aligned(y, 16)) return BS_ERR_ALIGNMENT;
+  const int m = stack->m, d = stack->d;
+  if (n_loaded == 0) return cuda_status(cudaMemsetAsync(y, 0, static_cast<size_t>(batch) * m * 2, stream));
+
+  if (batch <= kDecodeMaxBatch) {
+    const DecodeWs L = decode_ws_layout(m, d, n_loaded, batch);
+    if (workspace == nullptr || workspace_bytes < L.total) return BS_ERR_CAPACITY;
+    if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    DecodeParams p{};
+    p.blocks = stack->blocks;
+    p.block_bytes = stack->block_bytes;
+    p.x = x;
+    p.y = y;
+    p.inv_s = stack->inv_s;
+    p.vmax = stack->vmax;
+    p.zq = ws + L.zq;
+    p.csum = reinterpret_cast<float*>(ws + L.csum);
+    p.flags = reinterpret_cast<uint32_t*>(ws + L.flags);
+    p.part = reinterpret_cast<float*>(ws + L.part);
+    p.cnt = reinterpret_cast<unsigned long long*>(ws + L.cnt);
+    p.err = stack->err;
+    p.hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
+    p.m = m;
+    p.d = d;
+    p.n = n_loaded;
+    p.KG = d / kTileCols;
+    p.RT = m / kTileRows;
+    p.units = static_cast<long long>(p.RT) * n_loaded * p.KG;
+    p.stages = decode_pick_stages(batch);
+    p.x_bf16 = dt == BS_BF16 ? 1 : 0;
+    p.inject_unreachable = stack->inject_unreachable;
+    stack->inject_unreachable = 0;
+    p.timeout_ns = stack->timeout_ns;
+    long long grid = stack->sm_count < kMaxGrid ? stack->sm_count : kMaxGrid;
+    if (grid > p.units) grid = p.units;
+    return cuda_status(launch_decode(p, batch, static_cast<int>(grid), stack->sm_count, stream));
+  }
+
+  // prefill: W_hat tiles rebuilt in shared memory, tcgen05 GEMM
+  if (!stack->tmaps_ready) return BS_ERR_CUDA;
+  PrefillParams p{};
+  p.blocks = stack->blocks;
+  p.block_bytes = stack->block_bytes;
+  p.y = y;
+  p.inv_s = stack->inv_s;
+  p.err = stack->err;
+  p.m = m;
+  p.d = d;
+  p.n = n_loaded;
+  p.M = batch;
+  p.KG = d / kTileCols;
+  p.NT = batch >= 256 ? 256 : ((batch + 31) / 32) * 32;
+  p.timeout_ns = stack->timeout_ns;
+  const size_t limit = 227 * 1024;
+  int xs = 4, sb = 2;
+  while (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit && xs > 2) --xs;
+  if (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit) sb = 1;
+  while (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit && p.NT > 32) p.NT /= 2;
+  if (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit) return BS_ERR_CAPACITY;
+  p.xstages = xs;
+  p.sbufs = sb;
+  CUtensorMap tm_x;
+  const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t xstr[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t xbox[2] = {8, static_cast<cuuint32_t>(p.NT)};
+  if (!encode(&tm_x, dt == BS_BF16, 2, const_cast<void*>(x), xdims, xstr, xbox)) return BS_ERR_CUDA;
+  return cuda_status(launch_prefill(p, tm_x, stack->tm_u, stack->tm_v, dt == BS_BF16 ? 1 : 0, stream));
+}
+
+bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_stream_t stream) {
+  if (stack == nullptr || W_out == nullptr) return BS_ERR_INVALID_ARG;
+  if (dt != BS_F16 && dt != BS_BF16 && dt != BS_F32) return BS_ERR_INVALID_ARG;
+  if (n < 0 || n > stack->n_blocks) return BS_ERR_RANGE;
+  if (!aligned(W_out, 16)) return BS_ERR_ALIGNMENT;
+  const size_t elems = static_cast<size_t>(stack->m) * stack->d;
+  if (n == 0) return cuda_status(cudaMemsetAsync(W_out, 0, elems * (dt == BS_F32 ? 4 : 2), stream));
+  return cuda_status(
+      launch_reconstruct(stack->blocks, stack->block_bytes, stack->inv_s, stack->m, stack->d, n, W_out, dt, stream));
+}
+
+bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream) {
+  if (stack == nullptr || out == nullptr) return BS_ERR_INVALID_ARG;
+  if (block < 0 || block >= stack->n_blocks) return BS_ERR_RANGE;
+  return cuda_status(launch_unpack(stack->blocks + static_cast<size_t>(block) * stack->block_bytes, stack->m,
+                                   stack->d, out, stream));
+}
+
+bs_status bs_get_device_error(bs_stack_t stack) {
+  if (stack == nullptr) return BS_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, stack->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BS_ERR_CUDA;
+  if (v == 0) return BS_OK;
+  if (cudaMemset(stack->err, 0, sizeof(v)) != cudaSuccess) return BS_ERR_CUDA;
+  return (v & kErrTimeout) ? BS_ERR_TIMEOUT : BS_ERR_CUDA;
+}
+
+const char* bs_status_string(bs_status status) {
+  switch (status) {
+    case BS_OK: return "ok";
+    case BS_ERR_INVALID_ARG: return "invalid argument";
+    case BS_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need m % 128 == 0, d % 256 == 0, k == 16)";
+    case BS_ERR_ALIGNMENT: return "misaligned pointer";
+    case BS_ERR_CAPACITY: return "capacity or buffer size exceeded";
+    case BS_ERR_RANGE: return "block count or index out of range";
+    case BS_ERR_CUDA: return "CUDA error";
+    case BS_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case BS_ERR_NO_DEVICE: return "no usable sm_100 device";
+  }
+  return "unknown status";
+}
+
+bs_status bs_debug_set_wait(bs_stack_t stack, long long timeout_ns, int unreachable_flag) {
+  if (stack == nullptr || timeout_ns <= 0) return BS_ERR_INVALID_ARG;
+  stack->timeout_ns = static_cast<unsigned long long>(timeout_ns < 1000 ? 1000 : timeout_ns);
+  stack->inject_unreachable = unreachable_flag ? 1 : 0;
+  return BS_OK;
+}
+
+}  // extern "C"
