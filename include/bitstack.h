@@ -159,6 +159,22 @@ bs_status bs_drop_block(bs_stack_t stack);
 bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
                     void* workspace, size_t workspace_bytes, bs_stream_t stream);
 
+/* The same product as bs_linear for batch <= 4 (the decode path), for callers that
+ * cannot allocate device memory and so cannot pass a workspace: plugin hosts that
+ * give a kernel only its inputs and outputs, or serving loops that forbid
+ * allocation after start-up (cudaMalloc may synchronise the device or fail under
+ * memory pressure).  The pages have no counterpart to this call.
+ * The scratch is an 8 MiB array inside the library, held by every GPU that loads
+ * it until exit.  Calls whose scratch would exceed 8 MiB return BS_ERR_CAPACITY
+ * (e.g. 4096 x 4096, n = 8 needs 1.2 MiB at batch 1); batch > 4 returns
+ * BS_ERR_INVALID_ARG; the current device must be the stack's (BS_ERR_INVALID_ARG).
+ * The first call on each device looks up the array's device address and clears its
+ * header synchronously, so make it before any stream capture.  All calls on a device
+ * share the array: calls that can overlap on the GPU race; order them on one
+ * stream.  Allocates nothing.  Otherwise as bs_linear. */
+bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
+                             bs_stream_t stream);
+
 /* W_out = W_hat_n (m x d row-major, dtype BS_F32, BS_F16 or BS_BF16), for tests and
  * for users who want the dense weight (the unfused path of the restoration
  * snippet).  Asynchronous on `stream`. */

@@ -34,7 +34,7 @@ EXPORTS = (
     "bs_block_bytes", "bs_stack_device_bytes", "bs_workspace_bytes", "bs_pack_record",
     "bs_stack_create", "bs_stack_destroy", "bs_stack_num_blocks", "bs_append_block",
     "bs_drop_block", "bs_linear", "bs_reconstruct", "bs_unpack_signs",
-    "bs_get_device_error", "bs_status_string", "bs_debug_set_wait",
+    "bs_get_device_error", "bs_status_string", "bs_debug_set_wait", "bs_linear_no_alloc",
 )
 
 
@@ -65,6 +65,7 @@ def _load():
         "bs_get_device_error": (I, [P]),
         "bs_status_string": (ctypes.c_char_p, [I]),
         "bs_debug_set_wait": (I, [P, LL, I]),
+        "bs_linear_no_alloc": (I, [P, P, I, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -170,6 +171,13 @@ def bs_linear(handle: int, x, n_loaded: int, y, workspace=None, stream=None) -> 
     st = lib.bs_linear(handle, _ptr(x), x.shape[0], _dtype_code(x), n_loaded, _ptr(y), _ptr(workspace), ws_bytes,
                        _stream(stream))
     _check(st, "bs_linear")
+
+
+def bs_linear_no_alloc(handle: int, x, n_loaded: int, y, stream=None) -> None:
+    """bs_linear for batch <= 4 with the library's own fixed scratch array: for
+    callers that cannot allocate a workspace (see include/bitstack.h)."""
+    st = lib.bs_linear_no_alloc(handle, _ptr(x), x.shape[0], _dtype_code(x), n_loaded, _ptr(y), _stream(stream))
+    _check(st, "bs_linear_no_alloc")
 
 
 def bs_reconstruct(handle: int, n: int, W_out, stream=None) -> None:
