@@ -147,7 +147,9 @@ bs_status bs_drop_block(bs_stack_t stack);
 
 /* ----------------------------------------------------------------- compute ----- */
 
-/* y = x W_hat_n^T with n = n_loaded (0 <= n_loaded <= n_blocks).
+/* y = x W_hat_n^T with n = n_loaded (0 <= n_loaded <= n_blocks; the decode path
+ * takes up to 64 loaded blocks, the prefill path as many as its shared memory holds,
+ * BS_ERR_RANGE / BS_ERR_CAPACITY beyond).
  * x: batch x d row-major, y: batch x m row-major, both of dtype `dt` (BS_F16 or
  * BS_BF16), device pointers, 16-byte aligned.  n_loaded == 0 writes y = 0 (the
  * restoration accumulator starts at zero).  batch <= 4 runs the decode kernel (the

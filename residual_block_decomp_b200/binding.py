@@ -14,7 +14,8 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libbitstack_b200.so")
+# BITSTACK_LIB may name another build of the same ABI (e.g. a profiling build).
+LIB_PATH = os.environ.get("BITSTACK_LIB") or os.path.join(_PKG, "libbitstack_b200.so")
 
 BS_OK = 0
 BS_ERR_INVALID_ARG = 1

@@ -205,6 +205,7 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   if (n_loaded == 0) return cuda_status(cudaMemsetAsync(y, 0, static_cast<size_t>(batch) * m * 2, stream));
 
   if (batch <= kDecodeMaxBatch) {
+    if (n_loaded > kDecodeMaxBlocks) return BS_ERR_RANGE;
     const DecodeWs L = decode_ws_layout(m, d, n_loaded, batch);
     if (workspace == nullptr || workspace_bytes < L.total) return BS_ERR_CAPACITY;
     if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;

@@ -15,6 +15,7 @@ constexpr int kTileRows = 128;         // rows of a sign tile / an MMA M tile
 constexpr int kTileCols = 256;         // columns of a sign tile / one decode unit
 constexpr int kTileBytes = 4096;       // bytes of one sign tile
 constexpr int kDecodeMaxBatch = 4;     // batches up to this run the factored decode kernel
+constexpr int kDecodeMaxBlocks = 64;   // loaded blocks the decode kernel stages |V| maxima for
 constexpr int kMaxGrid = 160;          // cap on the decode kernel's persistent grid
 constexpr uint32_t kErrTimeout = 1u;   // device error word bit: a bounded wait ran out
 
