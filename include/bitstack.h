@@ -94,17 +94,20 @@ size_t bs_block_bytes(int m, int d, int k);
 
 /* Device bytes the caller must provide for a stack of `capacity_blocks` blocks:
  * capacity * bs_block_bytes (block i at offset i * bs_block_bytes) rounded up to
- * 256, plus a small metadata area (per-block column maxima of |V_i| and the device
- * error word).  0 on invalid arguments. */
+ * 256, plus 256 bytes that hold the stack's device error word.  0 on invalid
+ * arguments. */
 size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks);
 
 /* Workspace bytes bs_linear needs for `n_loaded` blocks and `batch` rows (0 when the
- * call needs none).  The caller zeroes a workspace once before its first use (e.g.
- * cudaMemsetAsync); the library keeps it consistent afterwards: its first 256 bytes
- * hold a launch epoch that tags the flags and counters of each call, so no clearing
- * is needed between calls, and calls captured in a CUDA graph may be replayed.  One
- * workspace may serve any number of stacks whose calls are ordered on one stream;
- * calls that may overlap on the GPU need distinct workspaces. */
+ * call needs none): one partial output per (128-row tile, chunk group) and batch row,
+ * and one arrival counter per row tile (about m * d * n * batch / 256 bytes).  The
+ * caller zeroes a workspace once before its first use (e.g. cudaMemsetAsync); every
+ * call that completes leaves its counters at zero again, so no clearing is needed
+ * between calls, and calls captured in a CUDA graph may be replayed.  After a call
+ * that reported BS_ERR_TIMEOUT the counters may be left non-zero: zero the workspace
+ * again before reusing it.  One workspace may serve any number of stacks whose calls
+ * are ordered on one stream; calls that may overlap on the GPU need distinct
+ * workspaces. */
 size_t bs_workspace_bytes(int m, int d, int k, int n_loaded, int batch);
 
 /* ---------------------------------------------------------- host packing ------ */
@@ -157,7 +160,12 @@ bs_status bs_drop_block(bs_stack_t stack);
  * int8 tensor cores); larger batches run the prefill kernel (W_hat tiles rebuilt in
  * shared memory, then a tcgen05 GEMM).  workspace: >= bs_workspace_bytes(m, d, k,
  * n_loaded, batch) device bytes, 256-aligned, zeroed before its first use (may be
- * NULL when the size is 0).  Asynchronous on `stream`; capturable in a CUDA graph. */
+ * NULL when the size is 0).  Asynchronous on `stream`; capturable in a CUDA graph.
+ * The decode kernel is launched with programmatic dependent launch: it may start, and
+ * read the stack's block area, before the kernel ahead of it on `stream` has
+ * finished; it reads x and the scale vector and touches the workspace and y only
+ * after that kernel has completed.  The block area is written only by this
+ * library's own copies (bs_append_block), which a dependent launch never overtakes. */
 bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
                     void* workspace, size_t workspace_bytes, bs_stream_t stream);
 
@@ -168,10 +176,11 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
  * memory pressure).  The pages have no counterpart to this call.
  * The scratch is an 8 MiB array inside the library, held by every GPU that loads
  * it until exit.  Calls whose scratch would exceed 8 MiB return BS_ERR_CAPACITY
- * (e.g. 4096 x 4096, n = 8 needs 1.2 MiB at batch 1); batch > 4 returns
+ * (e.g. 4096 x 4096, n = 8 needs 0.5 MiB at batch 1); batch > 4 returns
  * BS_ERR_INVALID_ARG; the current device must be the stack's (BS_ERR_INVALID_ARG).
- * The first call on each device looks up the array's device address and clears its
- * header synchronously, so make it before any stream capture.  All calls on a device
+ * The first call on each device looks up the array's device address synchronously,
+ * so make it before any stream capture; after bs_get_device_error has reported an
+ * error on a stack, the next call on that stack clears the array first.  All calls on a device
  * share the array: calls that can overlap on the GPU race; order them on one
  * stream.  Allocates nothing.  Otherwise as bs_linear. */
 bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
@@ -196,9 +205,10 @@ const char* bs_status_string(bs_status status);
 
 /* Sets the bound (nanoseconds) on every device-side wait of this stack's kernels
  * (default 500 ms; values < 1000 are raised to 1000).  With `unreachable_flag`
- * non-zero, the next bs_linear decode call waits for an activation-chunk flag
- * that no CTA ever sets, so its waits run out: a host-side way to exercise the
- * timeout path without faulting the GPU. */
+ * non-zero, the next bs_linear decode call leaves out the first sign-tile copy of
+ * every CTA, so the waits for it (and everything behind them) run out: a host-side
+ * way to exercise the timeout path without faulting the GPU.  Zero the workspace
+ * before reusing it after that call. */
 bs_status bs_debug_set_wait(bs_stack_t stack, long long timeout_ns, int unreachable_flag);
 
 #ifdef __cplusplus

@@ -17,9 +17,8 @@ bool gpu_shape_ok(int m, int d, int k) {
          d % kTileCols == 0;
 }
 
-size_t meta_bytes(int capacity) {
-  return align_up(static_cast<size_t>(capacity) * kK * sizeof(float) + 256, 256);
-}
+// After the block area: the stack's device error word (256 bytes reserved).
+size_t meta_bytes(int /*capacity*/) { return 256; }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -148,14 +147,13 @@ bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_bl
   s->block_bytes = bs_block_bytes(m, d, k);
   s->dev_bytes = dev_bytes;
   s->inv_s = dev_inv_scale;
-  s->vmax = reinterpret_cast<float*>(s->blocks + align_up(static_cast<size_t>(capacity_blocks) * s->block_bytes, 256));
-  s->err = reinterpret_cast<uint32_t*>(s->vmax + static_cast<size_t>(capacity_blocks) * kK);
+  s->err = reinterpret_cast<uint32_t*>(s->blocks + align_up(static_cast<size_t>(capacity_blocks) * s->block_bytes, 256));
   s->device = dev;
   s->sm_count = sms;
   s->timeout_ns = 500000000ull;
   s->inject_unreachable = 0;
   s->tmaps_ready = build_factor_maps(s) ? 1 : 0;
-  const cudaError_t e = cudaMemsetAsync(s->vmax, 0, meta_bytes(capacity_blocks), stream);
+  const cudaError_t e = cudaMemsetAsync(s->err, 0, meta_bytes(capacity_blocks), stream);
   if (e != cudaSuccess) {
     delete s;
     return BS_ERR_CUDA;
@@ -180,9 +178,7 @@ bs_status bs_append_block(bs_stack_t stack, const void* host_record, bs_stream_t
   if (stack == nullptr || host_record == nullptr) return BS_ERR_INVALID_ARG;
   if (stack->n_blocks >= stack->capacity) return BS_ERR_CAPACITY;
   uint8_t* slot = stack->blocks + static_cast<size_t>(stack->n_blocks) * stack->block_bytes;
-  cudaError_t e = cudaMemcpyAsync(slot, host_record, stack->block_bytes, cudaMemcpyDefault, stream);
-  if (e != cudaSuccess) return BS_ERR_CUDA;
-  e = launch_vmax(slot, stack->m, stack->d, stack->vmax + static_cast<size_t>(stack->n_blocks) * kK, stream);
+  const cudaError_t e = cudaMemcpyAsync(slot, host_record, stack->block_bytes, cudaMemcpyDefault, stream);
   if (e != cudaSuccess) return BS_ERR_CUDA;
   stack->n_blocks += 1;
   return BS_OK;
@@ -216,28 +212,24 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
     p.x = x;
     p.y = y;
     p.inv_s = stack->inv_s;
-    p.vmax = stack->vmax;
-    p.zq = ws + L.zq;
-    p.csum = reinterpret_cast<float*>(ws + L.csum);
-    p.flags = reinterpret_cast<uint32_t*>(ws + L.flags);
     p.part = reinterpret_cast<float*>(ws + L.part);
-    p.cnt = reinterpret_cast<unsigned long long*>(ws + L.cnt);
+    p.cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
     p.err = stack->err;
-    p.hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
     p.m = m;
     p.d = d;
     p.n = n_loaded;
     p.KG = d / kTileCols;
     p.RT = m / kTileRows;
-    p.units = static_cast<long long>(p.RT) * n_loaded * p.KG;
-    p.stages = decode_pick_stages(batch);
+    p.NCB = decode_groups_per_block(d, batch);
+    const long long segs = static_cast<long long>(p.RT) * n_loaded * p.NCB;
+    if (segs > (1ll << 30)) return BS_ERR_UNSUPPORTED_SHAPE;
+    p.segs = static_cast<int>(segs);
     p.x_bf16 = dt == BS_BF16 ? 1 : 0;
     p.inject_unreachable = stack->inject_unreachable;
     stack->inject_unreachable = 0;
     p.timeout_ns = stack->timeout_ns;
-    long long grid = stack->sm_count < kMaxGrid ? stack->sm_count : kMaxGrid;
-    if (grid > p.units) grid = p.units;
-    return cuda_status(launch_decode(p, batch, static_cast<int>(grid), stack->sm_count, stream));
+    const int grid = segs < stack->sm_count ? static_cast<int>(segs) : stack->sm_count;
+    return cuda_status(launch_decode(p, batch, grid, stream));
   }
 
   // prefill: W_hat tiles rebuilt in shared memory, tcgen05 GEMM
@@ -294,6 +286,7 @@ bs_status bs_get_device_error(bs_stack_t stack) {
   uint32_t v = 0;
   if (cudaMemcpy(&v, stack->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BS_ERR_CUDA;
   if (v == 0) return BS_OK;
+  stack->scratch_dirty = 1;
   if (cudaMemset(stack->err, 0, sizeof(v)) != cudaSuccess) return BS_ERR_CUDA;
   return (v & kErrTimeout) ? BS_ERR_TIMEOUT : BS_ERR_CUDA;
 }

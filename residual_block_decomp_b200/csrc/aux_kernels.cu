@@ -86,36 +86,6 @@ __global__ void unpack_kernel(const uint32_t* words, int m, int d, int8_t* out) 
   }
 }
 
-__global__ void __launch_bounds__(256) vmax_kernel(const __half* V, int d, float* out16) {
-  __shared__ float red[256 / 32][kK];
-  float mx[kK];
-#pragma unroll
-  for (int j = 0; j < kK; ++j) mx[j] = 0.0f;
-  for (int c = threadIdx.x; c < d; c += 256) {
-    const uint4 a = *reinterpret_cast<const uint4*>(V + static_cast<size_t>(c) * kK);
-    const uint4 b = *reinterpret_cast<const uint4*>(V + static_cast<size_t>(c) * kK + 8);
-    const __half* ha = reinterpret_cast<const __half*>(&a);
-    const __half* hb = reinterpret_cast<const __half*>(&b);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      mx[j] = fmaxf(mx[j], fabsf(__half2float(ha[j])));
-      mx[j + 8] = fmaxf(mx[j + 8], fabsf(__half2float(hb[j])));
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kK; ++j) {
-    float v = mx[j];
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5][j] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < kK) {
-    float v = 0.0f;
-    for (int w = 0; w < 256 / 32; ++w) v = fmaxf(v, red[w][threadIdx.x]);
-    out16[threadIdx.x] = v;
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_reconstruct(const uint8_t* blocks, unsigned long long block_bytes, const float* inv_s, int m,
@@ -129,13 +99,6 @@ cudaError_t launch_unpack(const uint8_t* record, int m, int d, int8_t* out, cuda
   const size_t total = static_cast<size_t>(m) * d;
   const int blocks = static_cast<int>((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
   unpack_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(record), m, d, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_vmax(const uint8_t* record, int m, int d, float* out16, cudaStream_t stream) {
-  const __half* V = reinterpret_cast<const __half*>(record + static_cast<size_t>(m) * d / 8 +
-                                                    static_cast<size_t>(2) * kK * m);
-  vmax_kernel<<<1, 256, 0, stream>>>(V, d, out16);
   return cudaGetLastError();
 }
 

@@ -11,21 +11,31 @@
 // N = 16 * batch columns per block.
 //
 // How it maps to sm_100a:
-//  * Z_i is quantised to two int8 planes (hi, lo) per column with a per-column scale
-//    sigma = max_c|x'[b,c]| * max_c|V_i[c,j]| / 127, so S_i Z_i runs on the int8 tensor
-//    cores (tcgen05.mma kind::i8) with exact int32 accumulation.  S = 1 - 2 Sb with
-//    Sb in {0, 1} the stored bit; the 1 part is a column sum added in the epilogue.
-//  * Sign bits are expanded in registers straight into u8 operands: one AND (and a
-//    shift for G < 8) per 4 columns gives bytes {0, 2^g}, g = K-step mod G; each g has
-//    its own TMEM accumulator and the epilogue recombines them exactly in int32.  The
-//    expanded A operand goes to tensor memory (tcgen05.st), never to shared memory.
-//  * One persistent launch: CTA c first quantises its share of the (block, 256-column)
-//    activation chunks and publishes each with an epoch flag; then it walks a
-//    contiguous range of units (row tile, block, 256-column group) in stream-K order:
-//    sign tiles (4 KiB) and activation chunks arrive by bulk copies into a ring of
-//    shared-memory stages, four warps expand signs into TMEM, one thread issues MMAs.
-//    Row tiles split across CTAs are reduced in fixed CTA order by the last CTA to
-//    arrive (an epoch-tagged counter), so results are deterministic.
+//  * Work is cut into segments: one 128-row tile of one block times C consecutive
+//    256-column chunks (C = 4 for one row of x, 2 for more).  Segments are numbered
+//    chunk-group-major (s = cg * RT + rt) and every CTA of the persistent grid takes
+//    a contiguous run of them, so a CTA touches one or two chunk groups.
+//  * Each CTA quantises the activation chunks of its own chunk groups (no exchange
+//    between CTAs): Z = (x / s) (.) V for the group's columns, per column (b, j) a
+//    step sigma = max |Z| / 32512 over the group, q = rint(Z / sigma) split exactly
+//    into two int8 planes q = 256 hi + lo.  So S_i Z_i runs on the int8 tensor cores
+//    (tcgen05.mma kind::i8) with exact int32 accumulation.  S = 1 - 2 Sb with Sb in
+//    {0, 1} the stored bit; the 1 part is the group's column sum, added in the epilogue.
+//  * Sign tiles (4 KiB per 128 x 256 unit, contiguous along a segment) stream from HBM
+//    by one 1-D bulk copy per segment into a ring of shared-memory stages, issued from
+//    the first instruction on.  Four warps expand sign bits in registers into u8
+//    operands (one AND, plus a shift when G < 8, per 4 columns: bytes {0, 2^g} for
+//    K-step t with g = t mod G; each g has its own TMEM accumulator and the epilogue
+//    recombines them exactly in int32) and store them to tensor memory (tcgen05.st).
+//    Up to four threads in four warps issue the MMAs; accumulators are double
+//    buffered so the epilogue of one segment overlaps the MMAs of the next.
+//  * The epilogue (four more warps) turns a segment's accumulators into one partial
+//    output per row and batch row.  When a CTA is done it counts its segments into
+//    per-row-tile counters; the CTA that completes a row tile sums its partials in
+//    fixed chunk-group order (deterministic) and resets the counter.
+//  * The launch allows programmatic dependent launch: the prologue (barriers, TMEM,
+//    the first sign copies, V rows) runs before the previous kernel in the stream has
+//    finished; x, s, the workspace and y are touched only after griddepcontrol.wait.
 //  * Every wait is bounded; a wait that runs out sets the device error word, and the
 //    CTA drains its copies and MMAs, frees tensor memory and returns.
 #include <cuda_bf16.h>
@@ -37,85 +47,83 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 288;
-constexpr int kWarpIss0 = 4;   // warps 4..7: MMA issuers (lane 0 each)
-constexpr int kWarpZ = 8;      // activation-chunk copies; allocates TMEM
-constexpr int kABufs = 4;      // A-operand buffers in TMEM (64 columns each, from column 256)
+constexpr int kThreads = 416;   // 13 warps
+constexpr int kWarpEpi0 = 4;    // warps 4..7: epilogue and activation-chunk production
+constexpr int kWarpIss0 = 8;    // warps 8..11: MMA issuers (lane 0 each)
+constexpr int kWarpCopy = 12;   // sign-tile copies; allocates TMEM
+constexpr int kABufs = 4;       // A-operand buffers in TMEM (64 columns each, from column 256): two pairs
 constexpr uint32_t kAcol0 = 256;
-constexpr int kBarExp = 1;     // named barrier: the four expander warps (128 threads)
-constexpr int kBarA = 2;       // named barrier: expander + issuer warps (256 threads), phase A
-constexpr int kMaxBlocks = kDecodeMaxBlocks;  // blocks whose |V| column maxima are staged in smem
-// Sign tiles stream through shared memory by per-thread 16-byte asynchronous copies
-// (each expander thread copies and later reads only its own row's 32 bytes), kSignAhead
-// units ahead, one commit group per unit (at most 8 groups outstanding per thread).
-// 1-D bulk copies of 4-16 KiB moved far less than HBM bandwidth here.
-constexpr int kSignAhead = 8;
-// Activation chunks come from L2 by 1-D bulk copies (the TMA engine), in groups of
-// consecutive units of one segment (contiguous in memory).  Keeping them off the
-// load/store path matters: behind the HBM-latency sign copies on that path, these L2
-// hits waited microseconds.
-__host__ __device__ constexpr int zgroup(int B) { return B == 1 ? 2 : 1; }       // units per chunk copy
-__host__ __device__ constexpr int zstages(int B) { return B == 1 ? 4 : (B == 2 ? 4 : (B == 3 ? 3 : 2)); }
+constexpr int kMaxStages = 16;
+constexpr int kBarEpi = 2;      // named barrier: warps 4-7
+constexpr int kBarA0 = 3;       // named barriers 3, 4: expanders + issuers, A-buffer pair g & 1
+constexpr int kBarAcc0 = 5;     // named barriers 5, 6: epilogue + issuers, accumulator j & 1
+constexpr int kGroup = 2;       // units per A-buffer pair (the hand-over granularity)
+static_assert(2 * kGroup == kABufs, "two A-buffer pairs");
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kSetHdr = 512;    // per chunk-group set: sigma_lo[64], column sums[64]
+constexpr int kURing = 4;       // U tiles (4 KiB each) in flight ahead of the epilogue
 
 struct Ctl {
-  uint64_t afull[kABufs], aempty[kABufs], accfull, accempty, drain[4];
+  uint64_t sfull[kMaxStages], sempty[kMaxStages];
+  uint64_t ufull[kURing];
+  uint64_t aempty[2];   // A-buffer pair free again: the MMAs that read it completed
+  uint64_t accfull[2], zfull[2], drain[4];
+  uint64_t vfull, xfull;  // inputs of the first chunk group: V rows; x rows and 1/s
   uint32_t tmem_base;
-  uint32_t tag, wait_tag, epoch;
   int abort;
-  int is_last;
-  float amax[kDecodeMaxBatch];
-  float cseg[16 * kDecodeMaxBatch];
-  float sig_lo[16 * kDecodeMaxBatch];
-  int zsum[16 * kDecodeMaxBatch];
-  float vmax[kMaxBlocks * kK];
+  int abort_snap;
+  int red_ok;
+  int amaxi[16 * kDecodeMaxBatch];   // max |Z| per column (float bits; values >= 0)
+  int zsum[16 * kDecodeMaxBatch];    // sum of q per column
 };
 
-// Shared-memory carve-up:
-//   [kSignAhead sign slots of 4 KiB][zstages activation stages][phase-A scratch]
-//   [barriers][Ctl];  activation stage = [chunk ZB][column sums 64 B per batch row]
-constexpr int kScratchBytes = kTileCols * kK * 2 + kTileCols * kDecodeMaxBatch * 4;  // V chunk + x' chunk
-__host__ __device__ constexpr int zstage_bytes(int B) {
-  return (zgroup(B) * (32 * B * kTileCols + 64 * B) + 127) / 128 * 128;
-}
-// Units [u, end) of the group that starts at unit u: at most `gs` units, never past
-// the end of u's segment (same row tile and block) or of the CTA's range.
-__device__ __forceinline__ int group_len(long long u, long long u1, int KG, int gs) {
-  const int kg = static_cast<int>(u % KG);  // per_rt is a multiple of KG
-  long long end = u - kg + KG;
-  if (end > u1) end = u1;
-  const long long len = end - u;
-  return static_cast<int>(len < gs ? len : gs);
+template <int B>
+struct Cfg {
+  static constexpr int NB = 32 * B;                 // MMA N: [hi plane 16B | lo plane 16B]
+  static constexpr int ZB = NB * kTileCols;         // operand bytes of one chunk
+  static constexpr int G = B == 1 ? 4 : (B == 2 ? 2 : 1);
+  static constexpr int NI = G < 4 ? G : 4;          // issuer w owns groups g with g % NI == w
+  static constexpr int C = decode_chunks_per_segment(B);
+  static constexpr int COLS = C * kTileCols;        // columns of a chunk group
+  static constexpr int SET = kSetHdr + C * ZB;      // one chunk-group set
+  static constexpr int VSCR = COLS * kK * 2;        // V rows of a group (fp16)
+  static constexpr int XSCR = COLS * B * 2 + COLS * 4;   // x rows (fp16/bf16), then 1/s (fp32)
+  static constexpr int URING = kURing * kTileBytes; // U rows of a row tile (128 x 16 fp16) per slot
+  static constexpr int STAGE = C * kTileBytes;
+  static constexpr int CTL = static_cast<int>((sizeof(Ctl) + 127) / 128 * 128);
+  static constexpr int FIXED = 2 * SET + VSCR + XSCR + URING + CTL;
+  static constexpr int NS0 = (kSmemLimit - FIXED) / STAGE;
+  static constexpr int NS = NS0 < kMaxStages ? NS0 : kMaxStages;
+  static constexpr int SMEM = NS * STAGE + FIXED;
+  static_assert(NS >= 2, "sign ring too small");
+  static_assert(2 * G * NB <= static_cast<int>(kAcol0), "accumulators must fit below the A buffers");
+  static_assert(XSCR % 128 == 0 && VSCR % 128 == 0, "scratch alignment");
+};
+
+struct Seg {
+  int i, rt, kgA, len, cg;
+};
+__device__ __forceinline__ Seg seg_of(int s, const DecodeParams& p, int C) {
+  Seg g;
+  g.cg = s / p.RT;
+  g.rt = s - g.cg * p.RT;
+  g.i = g.cg / p.NCB;
+  g.kgA = (g.cg - g.i * p.NCB) * C;
+  g.len = min(C, p.KG - g.kgA);
+  return g;
 }
 
-__device__ __forceinline__ void exp_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarExp), "n"(128) : "memory"); }
-__device__ __forceinline__ void phase_a_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarA), "n"(256) : "memory"); }
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 __device__ __forceinline__ void store_y(void* y, int bf16, size_t idx, float v) {
   if (bf16) static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
   else static_cast<__half*>(y)[idx] = __float2half_rn(v);
 }
-__device__ __forceinline__ void unpack8(const uint4& v, int bf16, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    if (bf16) {
-      const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-      f[2 * e] = __bfloat162float(h.x);
-      f[2 * e + 1] = __bfloat162float(h.y);
-    } else {
-      const __half2 h = *reinterpret_cast<const __half2*>(&w[e]);
-      f[2 * e] = __half2float(h.x);
-      f[2 * e + 1] = __half2float(h.y);
-    }
-  }
-}
-// Per-column quantisation step of the activation chunks: z ~ sigma_lo * q with
-// |q| <= 127 * 256, split exactly into q = 256 * hi + lo, hi in [-127, 127],
-// lo in [-128, 127]; so sigma_hi = 256 * sigma_lo.  The producer of a chunk and every
-// consumer evaluate the same expression, so they agree bit for bit.
-__device__ __forceinline__ float sigma_lo_of(float amax, float vmax) {
-  const float s = __fmul_rn(__fmul_rn(amax, vmax), 1.0f / 32512.0f);
-  return s > 0.0f ? s : 1.0f;
+__device__ __forceinline__ float x_at(const uint16_t* xr, int bf16, int idx) {
+  const uint16_t h = xr[idx];
+  return bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
 }
 
 __device__ __forceinline__ void set_error(const DecodeParams& p, Ctl* ctl) {
@@ -123,543 +131,585 @@ __device__ __forceinline__ void set_error(const DecodeParams& p, Ctl* ctl) {
   atomicOr(p.err, kErrTimeout);
 }
 
-// CTA owning unit u under the split u0(c) = floor(c U / grid).
-__device__ __forceinline__ int cta_of(long long u, long long U, int grid) {
-  return static_cast<int>(((u + 1) * grid + U - 1) / U) - 1;
+// Byte addresses of a chunk group's inputs in the stack and in x.
+__device__ __forceinline__ const uint8_t* v_rows(const DecodeParams& p, const Seg& sg) {
+  return p.blocks + static_cast<size_t>(sg.i) * p.block_bytes + static_cast<size_t>(p.m) * p.d / 8 +
+         static_cast<size_t>(2) * kK * p.m + static_cast<size_t>(sg.kgA) * kTileCols * kK * 2;
+}
+__device__ __forceinline__ const uint8_t* u_tile(const DecodeParams& p, int i, int rt) {
+  return p.blocks + static_cast<size_t>(i) * p.block_bytes + static_cast<size_t>(p.m) * p.d / 8 +
+         static_cast<size_t>(rt) * kTileRows * kK * 2;
 }
 
-template <int B, int G>
+// Loads the inputs of chunk group `sg` into the scratch with plain loads (the later
+// groups of a CTA; the first one arrives by bulk copies).  Called by the 128 epilogue
+// threads after griddep_wait.
+template <int B>
+__device__ void load_set_inputs(const DecodeParams& p, uint8_t* vscr, uint8_t* xscr, const Seg& sg, int tid) {
+  using K = Cfg<B>;
+  const int cols = sg.len * kTileCols, col0 = sg.kgA * kTileCols;
+  const uint4* vsrc = reinterpret_cast<const uint4*>(v_rows(p, sg));
+  for (int v = tid; v < cols * 2; v += 128) reinterpret_cast<uint4*>(vscr)[v] = __ldg(vsrc + v);
+  uint16_t* xr = reinterpret_cast<uint16_t*>(xscr);
+  for (int idx = tid; idx < B * cols; idx += 128) {
+    const int b = idx / cols, c = idx - b * cols;
+    xr[b * K::COLS + c] = static_cast<const uint16_t*>(p.x)[static_cast<size_t>(b) * p.d + col0 + c];
+  }
+  float* isv = reinterpret_cast<float*>(xscr + K::COLS * B * 2);
+  for (int c = tid; c < cols; c += 128) isv[c] = __ldg(p.inv_s + col0 + c);
+}
+
+// Quantises the activation chunks of chunk group `sg` (inputs already in the scratch:
+// V rows, x rows, 1/s) into `set`: operand planes in the UMMA no-swizzle K-major
+// layout, the per-column step sigma_lo and the dequantised column sum.  Run by the
+// 128 epilogue threads, which share named barrier kBarEpi; it has no other wait, so
+// every thread passes the same barriers.  `zfull` is signalled unless `skip`.
+template <int B>
+__device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xscr, int bf16, Ctl* ctl, const Seg& sg,
+                            int tid, uint64_t* zfull, bool skip) {
+  using K = Cfg<B>;
+  constexpr int NT = 128;
+  const int cols = sg.len * kTileCols;
+  const __half* vh = reinterpret_cast<const __half*>(vscr);
+  const uint16_t* xr = reinterpret_cast<const uint16_t*>(xscr);
+  const float* isv = reinterpret_cast<const float*>(xscr + K::COLS * B * 2);
+  const int items = (cols / 16) * 16 * B;   // (16-column group, column (b, j)), column fastest
+  if (!skip) {
+    // pass 1: max |Z| per column over the group; a thread folds its items of one
+    // column before touching shared memory
+    int lcol = -1;
+    float lmx = 0.0f;
+    for (int it = tid; it < items; it += NT) {
+      const int c16 = it / (16 * B), col = it - c16 * 16 * B;
+      const int b = col >> 4, j = col & 15;
+      float mx = 0.0f;
+#pragma unroll
+      for (int kin = 0; kin < 16; ++kin) {
+        const int c = c16 * 16 + kin;
+        const float xs = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
+        mx = fmaxf(mx, fabsf(__fmul_rn(xs, __half2float(vh[c * kK + j]))));
+      }
+      if (col != lcol) {
+        if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
+        lcol = col;
+        lmx = mx;
+      } else {
+        lmx = fmaxf(lmx, mx);
+      }
+    }
+    if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
+  }
+  named_sync(kBarEpi, NT);
+  if (!skip) {
+    // pass 2: q = rint(Z / sigma_lo), |q| <= 127 * 256, q = 256 hi + lo
+    uint8_t* ops = set + kSetHdr;
+    int lcol = -1, lsum = 0;
+    float slo = 1.0f, rlo = 1.0f;
+    for (int it = tid; it < items; it += NT) {
+      const int c16 = it / (16 * B), col = it - c16 * 16 * B;
+      const int b = col >> 4, j = col & 15;
+      if (col != lcol) {
+        if (lcol >= 0) atomicAdd(&ctl->zsum[lcol], lsum);
+        lcol = col;
+        lsum = 0;
+        const float amax = __int_as_float(ctl->amaxi[col]);
+        slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
+        rlo = 1.0f / slo;
+      }
+      uint32_t hw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int kin = 0; kin < 16; ++kin) {
+        const int c = c16 * 16 + kin;
+        const float xs = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
+        const float z = __fmul_rn(xs, __half2float(vh[c * kK + j]));
+        int qv = __float2int_rn(z * rlo);
+        qv = max(-32512, min(32512, qv));
+        const int qh = (qv + 128) >> 8;
+        const int ql = qv - (qh << 8);
+        lsum += qv;
+        hw[kin >> 2] |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * (kin & 3));
+        lw[kin >> 2] |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * (kin & 3));
+      }
+      // chunk cc, K-step t (32 columns), K half kc, 8-row core matrix n / 8
+      const int cc = c16 >> 4, g16 = c16 & 15;
+      const int t = g16 >> 1, kc = g16 & 1;
+      const int nh = col, nl = 16 * B + col;
+      uint8_t* base = ops + static_cast<size_t>(cc) * K::ZB;
+      *reinterpret_cast<uint4*>(base + ((t * (K::NB / 8) + nh / 8) * 2 + kc) * 128 + (nh % 8) * 16) =
+          make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(base + ((t * (K::NB / 8) + nl / 8) * 2 + kc) * 128 + (nl % 8) * 16) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    if (lcol >= 0) atomicAdd(&ctl->zsum[lcol], lsum);
+    fence_proxy_async_smem();   // the MMAs read the operands through the async proxy
+  }
+  named_sync(kBarEpi, NT);
+  if (tid < 16 * B) {
+    if (!skip) {
+      const float amax = __int_as_float(ctl->amaxi[tid]);
+      const float slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
+      float* hdr = reinterpret_cast<float*>(set);
+      hdr[tid] = slo;
+      hdr[64 + tid] = __fmul_rn(slo, static_cast<float>(ctl->zsum[tid]));
+    }
+    ctl->amaxi[tid] = 0;
+    ctl->zsum[tid] = 0;
+  }
+  named_sync(kBarEpi, NT);
+  if (tid == 0 && !skip) mbar_arrive(zfull);
+}
+
+template <int B>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
-  constexpr int NB = 32 * B;                 // MMA N: [hi plane 16B | lo plane 16B]
-  constexpr int ZB = NB * kTileCols;         // bytes of one activation chunk
-  constexpr int CB = 64 * B;                 // bytes of one chunk's column sums
-  constexpr int ZST = zstage_bytes(B);
-  constexpr int ZS = zstages(B);
-  constexpr int GZ = zgroup(B);
-  constexpr int NI = G < 4 ? G : 4;          // MMA issuers: issuer w owns groups g with g % NI == w
+  using K = Cfg<B>;
+  constexpr int NB = K::NB, G = K::G, NI = K::NI, C = K::C, NS = K::NS;
   constexpr uint32_t IDESC = make_idesc(2u, 0u, 1u, 128u, NB);  // s32 <- u8 x s8, M=128, N=NB
-  static_assert(G * NB <= 256, "accumulators must fit below the A buffers");
 
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* zst_base = smem + kSignAhead * kTileBytes;
-  uint8_t* scratch = zst_base + ZS * ZST;
-  uint64_t* zfull = reinterpret_cast<uint64_t*>(scratch + kScratchBytes);
-  uint64_t* zempty = zfull + ZS;
-  Ctl* ctl = reinterpret_cast<Ctl*>(zempty + ZS);
+  uint8_t* stages = smem;
+  uint8_t* sets = smem + NS * K::STAGE;
+  uint8_t* vscr = sets + 2 * K::SET;
+  uint8_t* xscr = vscr + K::VSCR;
+  uint8_t* uring = xscr + K::XSCR;
+  Ctl* ctl = reinterpret_cast<Ctl*>(uring + K::URING);
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x, grid = gridDim.x;
-  const long long U = p.units;
-  const long long u0 = static_cast<long long>(cta) * U / grid;
-  const long long u1 = static_cast<long long>(cta + 1) * U / grid;
-  const int KG = p.KG;
-  const int per_rt = p.n * KG;
+  const int s0 = static_cast<int>(static_cast<long long>(cta) * p.segs / grid);
+  const int s1 = static_cast<int>(static_cast<long long>(cta + 1) * p.segs / grid);
+  const int nseg = s1 - s0;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
-  const size_t sign_bytes = static_cast<size_t>(p.m) * p.d / 8;
+  const int NC = p.n * p.NCB;   // chunk groups = partials per row tile
+  const Seg sg0 = seg_of(s0, p, C);
 
-  // Expander threads start streaming their sign rows before anything else.
-  auto sign_src = [&](long long u) {
-    const long long rt = u / per_rt, rem = u % per_rt;
-    const int i = static_cast<int>(rem / KG), kg = static_cast<int>(rem % KG);
-    return p.blocks + static_cast<size_t>(i) * p.block_bytes + (static_cast<size_t>(rt) * KG + kg) * kTileBytes;
-  };
-  if (warp < 4) {
-    for (int j = 0; j < kSignAhead; ++j) {
-      if (u0 + j < u1) {
-        const uint8_t* src = sign_src(u0 + j);
-        uint8_t* dst = smem + j * kTileBytes;
-        cp_async16(dst + threadIdx.x * 16, src + threadIdx.x * 16);
-        cp_async16(dst + 2048 + threadIdx.x * 16, src + 2048 + threadIdx.x * 16);
+  griddep_launch_dependents();
+
+  // ------------------------------------------------------------------ set-up -----
+  int issued = 0;   // sign copies issued (copy warp, lane 0)
+  if (warp == kWarpCopy) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    if (lane == 0) {
+      for (int s = 0; s < kMaxStages; ++s) {
+        mbar_init(&ctl->sfull[s], 1);
+        mbar_init(&ctl->sempty[s], 4);
       }
-      cp_async_commit();
+      for (int u = 0; u < kURing; ++u) mbar_init(&ctl->ufull[u], 1);
+      for (int q = 0; q < 2; ++q) {
+        mbar_init(&ctl->aempty[q], NI);
+        mbar_init(&ctl->accfull[q], NI);
+        mbar_init(&ctl->zfull[q], 1);
+      }
+      for (int w = 0; w < 4; ++w) mbar_init(&ctl->drain[w], 1);
+      mbar_init(&ctl->vfull, 1);
+      mbar_init(&ctl->xfull, 1);
+      ctl->abort = 0;
+      for (int c = 0; c < 16 * kDecodeMaxBatch; ++c) {
+        ctl->amaxi[c] = 0;
+        ctl->zsum[c] = 0;
+      }
+      fence_barrier_init();
+      // Stack memory only, so these copies may start before the previous kernel in
+      // the stream has finished: V rows of the first chunk group, the first sign
+      // stages, the first U tiles.
+      if (nseg > 0) {
+        const uint32_t vb = static_cast<uint32_t>(sg0.len) * kTileCols * kK * 2;
+        mbar_arrive_expect_tx(&ctl->vfull, vb);
+        bulk_g2s(vscr, v_rows(p, sg0), vb, &ctl->vfull);
+      }
+      for (; issued < NS && issued < nseg; ++issued) {
+        if (p.inject_unreachable && issued == 0) continue;
+        const Seg sg = seg_of(s0 + issued, p, C);
+        const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
+        mbar_arrive_expect_tx(&ctl->sfull[issued], bytes);
+        bulk_g2s(stages + issued * K::STAGE,
+                 p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
+                     (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
+                 bytes, &ctl->sfull[issued]);
+      }
+      for (int j = 0; j < kURing && j < nseg; ++j) {
+        const Seg sg = seg_of(s0 + j, p, C);
+        mbar_arrive_expect_tx(&ctl->ufull[j], kTileBytes);
+        bulk_g2s(uring + j * kTileBytes, u_tile(p, sg.i, sg.rt), kTileBytes, &ctl->ufull[j]);
+      }
     }
   }
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < ZS; ++s) {
-      mbar_init(&zfull[s], 1);
-      mbar_init(&zempty[s], NI);
-    }
-    for (int a = 0; a < kABufs; ++a) {
-      mbar_init(&ctl->afull[a], 128);
-      mbar_init(&ctl->aempty[a], NI);
-    }
-    mbar_init(&ctl->accfull, NI);
-    mbar_init(&ctl->accempty, 128);
-    for (int w = 0; w < 4; ++w) mbar_init(&ctl->drain[w], 1);
-    ctl->abort = 0;
-    const uint32_t e = *reinterpret_cast<volatile uint32_t*>(p.hdr);
-    ctl->epoch = e;
-    ctl->tag = e + 1u;
-    ctl->wait_tag = p.inject_unreachable ? ((e + 1u) ^ 0x80000000u) : (e + 1u);
-    for (int i = 0; i < 16 * kDecodeMaxBatch; ++i) ctl->zsum[i] = 0;
-    for (int b = 0; b < kDecodeMaxBatch; ++b) ctl->amax[b] = 0.0f;
-    fence_barrier_init();
-  }
-  if (warp == kWarpZ) tmem_alloc(&ctl->tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const uint32_t tag = ctl->tag, wait_tag = ctl->wait_tag;
 
-  if (warp == kWarpZ) {
-    // ---------------------------------------------- activation-chunk producer -----
-    // All 32 lanes first wait, in parallel, for every chunk this CTA will read; then
-    // each chunk is copied by all lanes (16-byte cp.async), whose arrivals complete
-    // the stage's barrier.
-    const long long count = u1 - u0;
-    const int distinct = static_cast<int>(count < per_rt ? count : per_rt);
-    bool ok = true;
-    for (int idx = lane; idx < distinct && ok; idx += 32) {
-      const int q = static_cast<int>((u0 + idx) % per_rt);
-      while (ld_acquire_u32(p.flags + q) != wait_tag) {
-        if (*abort_flag || globaltimer_ns() > deadline) { ok = false; break; }
-        __nanosleep(32);
-      }
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok && lane == 0) set_error(p, ctl);
-    if (lane == 0) {
-      long long g = 0;
-      if (ok) {
-        fence_proxy_async_global();   // the chunks were written by generic stores
-        for (long long u = u0; u < u1; ++g) {
-          const int len = group_len(u, u1, KG, GZ);
-          const int s = static_cast<int>(g % ZS);
-          const long long ph = g / ZS;
-          if (ph > 0 && !mbar_wait(&zempty[s], static_cast<uint32_t>((ph - 1) & 1), deadline, abort_flag)) {
-            set_error(p, ctl);
-            break;
-          }
-          const int q = static_cast<int>(u % per_rt);  // chunk index i * KG + kg
-          uint8_t* st = zst_base + static_cast<size_t>(s) * ZST;
-          mbar_arrive_expect_tx(&zfull[s], static_cast<uint32_t>(len) * (ZB + CB));
-          bulk_g2s(st, p.zq + static_cast<size_t>(q) * ZB, static_cast<uint32_t>(len) * ZB, &zfull[s]);
-          bulk_g2s(st + GZ * ZB, p.csum + static_cast<size_t>(q) * 16 * B, static_cast<uint32_t>(len) * CB, &zfull[s]);
-          u += len;
-        }
-      }
-      const long long issued = g;
-      for (long long j = (issued > ZS ? issued - ZS : 0); j < issued; ++j)
-        mbar_wait(&zfull[j % ZS], static_cast<uint32_t>((j / ZS) & 1), globaltimer_ns() + 100000000ull, nullptr);
-    }
-  } else {
-    // --------- warps 0-7: phase A (quantise and publish the owned activation chunks) ---
-    const int ta = threadIdx.x;  // 0..255
-    const int chunks = p.n * KG;
-    // Inputs of the first chunk this CTA owns are loaded before the |x| scan so that
-    // both round trips to memory overlap.
-    uint4 vv0 = make_uint4(0, 0, 0, 0), vv1 = make_uint4(0, 0, 0, 0);
-    float xsv[B];
-    auto load_chunk = [&](int q) {
-      const int i = q / KG, c0 = (q % KG) * kTileCols;
-      const uint8_t* vsrc = p.blocks + static_cast<size_t>(i) * p.block_bytes + sign_bytes +
-                            static_cast<size_t>(2) * kK * p.m;
-      const uint4* v4 = reinterpret_cast<const uint4*>(vsrc + static_cast<size_t>(c0) * kK * 2);
-      vv0 = __ldg(v4 + ta);
-      vv1 = __ldg(v4 + ta + 256);                                              // 512 x 16 B = 8 KiB
-      const float is = __ldg(p.inv_s + c0 + ta);
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        const size_t xi = static_cast<size_t>(b) * p.d + c0 + ta;
-        const float xv = p.x_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.x)[xi])
-                                  : __half2float(static_cast<const __half*>(p.x)[xi]);
-        xsv[b] = __fmul_rn(xv, is);
-      }
+  if (warp < 4) {
+    // ------------------------------------------------ expanders (rows = lanes) -----
+    // Units are walked in order and handed to the issuers in pairs (A buffers
+    // 2 (g & 1) and 2 (g & 1) + 1) through named barrier kBarA0 + (g & 1), which the
+    // issuers also sync on, so neither side can run a generation ahead.  A thread
+    // whose wait ran out keeps walking in "failed" mode, skipping work but passing
+    // every named barrier; failure is decided per warp by vote.
+    const int tid = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    bool failed = false;
+    auto check = [&](bool ok) {
+      if (!__all_sync(0xffffffffu, ok)) failed = true;
     };
-    if (cta < chunks) load_chunk(cta);
-    {
-      for (int e = ta; e < p.n * kK && e < kMaxBlocks * kK; e += 256) ctl->vmax[e] = __ldg(p.vmax + e);
-      // max_c |x[b, c] / s_c| for every row b of x, 8 columns per load
-      float mx[B];
-#pragma unroll
-      for (int b = 0; b < B; ++b) mx[b] = 0.0f;
-      const int nvec = p.d / 8;
-      for (int v0 = ta; v0 < nvec; v0 += 256 * 2) {
-        uint4 xv[2][B];
-        float4 sv[2][2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int v = v0 + r * 256;
-          if (v < nvec) {
-            sv[r][0] = __ldg(reinterpret_cast<const float4*>(p.inv_s) + 2 * v);
-            sv[r][1] = __ldg(reinterpret_cast<const float4*>(p.inv_s) + 2 * v + 1);
-#pragma unroll
-            for (int b = 0; b < B; ++b)
-              xv[r][b] = __ldg(reinterpret_cast<const uint4*>(p.x) + static_cast<size_t>(b) * nvec + v);
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          if (v0 + r * 256 < nvec) {
-            const float is[8] = {sv[r][0].x, sv[r][0].y, sv[r][0].z, sv[r][0].w,
-                                 sv[r][1].x, sv[r][1].y, sv[r][1].z, sv[r][1].w};
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-              float f[8];
-              unpack8(xv[r][b], p.x_bf16, f);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) mx[b] = fmaxf(mx[b], fabsf(__fmul_rn(f[e], is[e])));
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        float v = mx[b];
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) atomicMax(reinterpret_cast<int*>(&ctl->amax[b]), __float_as_int(v));
-      }
-      phase_a_sync();
-    }
-    float amax[B];
-#pragma unroll
-    for (int b = 0; b < B; ++b) amax[b] = ctl->amax[b];
-    {
-      __half* vs = reinterpret_cast<__half*>(scratch);                       // [256][16]
-      float* xs = reinterpret_cast<float*>(scratch + kTileCols * kK * 2);     // [B][256]
-      for (int q = cta; q < chunks; q += grid) {
-        const int i = q / KG;
-        if (q != cta) load_chunk(q);
-        reinterpret_cast<uint4*>(vs)[ta] = vv0;
-        reinterpret_cast<uint4*>(vs)[ta + 256] = vv1;
-#pragma unroll
-        for (int b = 0; b < B; ++b) xs[b * kTileCols + ta] = xsv[b];
-        phase_a_sync();
-        uint8_t* zdst = p.zq + static_cast<size_t>(q) * ZB;
-        for (int it = ta; it < 16 * B * 16; it += 256) {
-          const int cg = it / (16 * B);          // 16-column group of the chunk
-          const int col = it % (16 * B);         // b * 16 + j
-          const int b = col / 16, j = col % 16;
-          const float slo = sigma_lo_of(amax[b], ctl->vmax[i * 16 + j]);
-          const float rlo = 1.0f / slo;
-          uint32_t hw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
-          int sq = 0;
-#pragma unroll
-          for (int kin = 0; kin < 16; ++kin) {
-            const int cl = cg * 16 + kin;
-            const float z = __fmul_rn(xs[b * kTileCols + cl], __half2float(vs[cl * kK + j]));
-            int qv = __float2int_rn(z * rlo);
-            qv = max(-32512, min(32512, qv));
-            const int qh = (qv + 128) >> 8;
-            const int ql = qv - (qh << 8);
-            sq += qv;
-            hw[kin >> 2] |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * (kin & 3));
-            lw[kin >> 2] |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * (kin & 3));
-          }
-          // B operand layout: K-step t (32 columns), 8-row group n/8, K half kc.
-          const int t = cg >> 1, kc = cg & 1;
-          const int nh = col, nl = 16 * B + col;
-          uint8_t* ph = zdst + ((t * (NB / 8) + nh / 8) * 2 + kc) * 128 + (nh % 8) * 16;
-          uint8_t* pl = zdst + ((t * (NB / 8) + nl / 8) * 2 + kc) * 128 + (nl % 8) * 16;
-          *reinterpret_cast<uint4*>(ph) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(pl) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          atomicAdd(&ctl->zsum[col], sq);
-        }
-        phase_a_sync();
-        if (ta < 16 * B) {
-          const int b = ta / 16, j = ta % 16;
-          const float slo = sigma_lo_of(amax[b], ctl->vmax[i * 16 + j]);
-          p.csum[static_cast<size_t>(q) * 16 * B + ta] = __fmul_rn(slo, static_cast<float>(ctl->zsum[ta]));
-          ctl->zsum[ta] = 0;
-        }
-        phase_a_sync();
-        if (ta == 0) {   // publish: every write of the chunk happens before the release
-          __threadfence();
-          st_release_u32(p.flags + q, tag);
-        }
-      }
-    }
-
-    if (warp >= kWarpIss0) {
-      // ---------------------------------------------------------- MMA issuers -----
-      const int w = warp - kWarpIss0;
-      if (lane == 0 && w < NI) {
-        long long k = 0;
-        int seg = 0;
-        bool issued_any = false;
-        long long zg = -1;   // chunk group of the current unit, its length and position
-        int zlen = 0, zpos = 0;
-        for (long long u = u0; u < u1; ++u, ++k) {
-          if (zpos == zlen) {
-            ++zg;
-            zpos = 0;
-            zlen = group_len(u, u1, KG, GZ);
-          }
-          const int zs = static_cast<int>(zg % ZS);
-          const uint32_t zph = static_cast<uint32_t>((zg / ZS) & 1);
-          const int a = static_cast<int>(k % kABufs);
-          const uint32_t pa = static_cast<uint32_t>((k / kABufs) & 1);
-          const int kg = static_cast<int>((u % per_rt) % KG);
-          const bool seg_start = (u == u0) || (kg == 0);
-          const bool seg_end = (u + 1 == u1) || (kg == KG - 1);
-          if (!mbar_wait(&zfull[zs], zph, deadline, abort_flag) ||
-              !mbar_wait(&ctl->afull[a], pa, deadline, abort_flag) ||
-              (seg_start && seg > 0 &&
-               !mbar_wait(&ctl->accempty, static_cast<uint32_t>((seg - 1) & 1), deadline, abort_flag))) {
-            set_error(p, ctl);
-            break;
-          }
-          tc_fence_after();
-          const uint32_t zaddr = smem_u32(zst_base + static_cast<size_t>(zs) * ZST + static_cast<size_t>(zpos) * ZB);
-          const uint32_t acol = kAcol0 + 64u * static_cast<uint32_t>(a);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int g = t % G;
-            if (g % NI != w) continue;
-            const uint64_t bdesc = smem_desc_noswizzle(zaddr + t * (NB / 8) * 256, 128, 256);
-            mma_i8_ts(tmem + g * NB, tmem + acol + 8 * t, bdesc, IDESC, (seg_start && t < G) ? 0u : 1u);
-          }
-          issued_any = true;
-          if (++zpos == zlen) tc_commit(&zempty[zs]);   // the group's chunks are consumed
-          tc_commit(&ctl->aempty[a]);
-          if (seg_end) {
-            tc_commit(&ctl->accfull);
-            ++seg;
-          }
-        }
-        if (issued_any) {
-          tc_commit(&ctl->drain[w]);
-          mbar_wait(&ctl->drain[w], 0, globaltimer_ns() + 100000000ull, nullptr);
-        }
-      }
-    } else {
-      // ------------------------------------------ warps 0-3: expand, epilogue -----
-      const int tid = threadIdx.x;  // 0..127 = row within the tile = TMEM lane
-      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-      // Control flow is uniform across the 128 threads: a thread whose wait ran out
-      // keeps walking the loop in "failed" mode, skipping work but passing every
-      // named barrier; each warp decides failure by vote so warp-collective tcgen05
-      // ops stay uniform.
-      float ypart[B];
-#pragma unroll
-      for (int b = 0; b < B; ++b) ypart[b] = 0.0f;
-      float cacc = 0.0f;  // column-sum accumulator of this segment (threads < 16B)
-      uint4 ua = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);   // this row of U_i
-      long long k = 0;
-      int seg = 0;
-      long long zg = -1;   // chunk group of the current unit, its length and position
-      int zlen = 0, zpos = 0;
-      bool failed = false;
-      auto check = [&](bool ok) {
-        if (!__all_sync(0xffffffffu, ok)) failed = true;
-      };
-      for (long long u = u0; u < u1; ++u, ++k) {
-        const bool new_zgroup = (zpos == zlen);
-        if (new_zgroup) {
-          ++zg;
-          zpos = 0;
-          zlen = group_len(u, u1, KG, GZ);
-        }
-        const int slot = static_cast<int>(k % kSignAhead);
-        const int zs = static_cast<int>(zg % ZS);
-        const uint32_t zph = static_cast<uint32_t>((zg / ZS) & 1);
-        const int a = static_cast<int>(k % kABufs);
-        const long long pa = k / kABufs;
-        const long long rt = u / per_rt, rem = u % per_rt;
-        const int i = static_cast<int>(rem / KG), kg = static_cast<int>(rem % KG);
-        const bool seg_start = (u == u0) || (kg == 0);
-        if (seg_start) {
-          cacc = 0.0f;
-          const uint8_t* urow = p.blocks + static_cast<size_t>(i) * p.block_bytes + sign_bytes +
-                                (static_cast<size_t>(rt) * kTileRows + tid) * kK * 2;
-          ua = __ldg(reinterpret_cast<const uint4*>(urow));
-          ub = __ldg(reinterpret_cast<const uint4*>(urow + 16));
-        }
-        // this unit's sign words (own row, own copies) and the next prefetch
-        cp_async_wait<kSignAhead - 1>();
-        uint8_t* sdst = smem + slot * kTileBytes;
-        const uint4 wa = *reinterpret_cast<const uint4*>(sdst + tid * 16);
-        const uint4 wb = *reinterpret_cast<const uint4*>(sdst + 2048 + tid * 16);
-        if (u + kSignAhead < u1) {
-          const uint8_t* src = sign_src(u + kSignAhead);
-          cp_async16(sdst + tid * 16, src + tid * 16);
-          cp_async16(sdst + 2048 + tid * 16, src + 2048 + tid * 16);
-        }
-        cp_async_commit();
-        const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    int j = 0, c = 0;
+    Seg sg = sg0;
+    for (int g = 0; j < nseg; ++g) {
+      const int half = g & 1;
+      if (!failed && g >= 2)
+        check(mbar_wait(&ctl->aempty[half], static_cast<uint32_t>(((g >> 1) - 1) & 1), deadline, abort_flag));
+      for (int q = 0; q < kGroup && j < nseg; ++q) {
+        const int st = j % NS;
+        if (c == 0 && !failed) check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
         if (!failed) {
-          if (new_zgroup) check(mbar_wait(&zfull[zs], zph, deadline, abort_flag));
-          if (!failed && tid < 16 * B)
-            cacc += reinterpret_cast<const float*>(zst_base + static_cast<size_t>(zs) * ZST + GZ * ZB)[zpos * 16 * B + tid];
-          if (!failed && pa > 0)
-            check(mbar_wait(&ctl->aempty[a], static_cast<uint32_t>((pa - 1) & 1), deadline, abort_flag));
-        }
-        if (!failed) {
-          const uint32_t abase = tmem + lane_base + kAcol0 + 64u * static_cast<uint32_t>(a);
+          const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
+          const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
+          const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
+          const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          const uint32_t abase = tmem + lane_base + kAcol0 + 64u * static_cast<uint32_t>(kGroup * half + q);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t r[32];
 #pragma unroll
             for (int tt = 0; tt < 4; ++tt) {
               const int t = 4 * h + tt;
-              const int g = t % G;
-              const uint32_t mask = 0x01010101u << g;
+              const int gg = t % G;
+              const uint32_t mask = 0x01010101u << gg;
 #pragma unroll
-              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (t - g)) & mask;
+              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (t - gg)) & mask;
             }
             tmem_st32(abase + 32 * h, r);
           }
-          tc_wait_st();
-          tc_fence_before();
-          mbar_arrive(&ctl->afull[a]);
         }
-        ++zpos;
-
-        const bool seg_end = (u + 1 == u1) || (kg == KG - 1);
-        if (seg_end) {
-          if (tid < 16 * B) {
-            const int b = tid / 16, j = tid % 16;
-            ctl->cseg[tid] = cacc;
-            ctl->sig_lo[tid] = sigma_lo_of(amax[b], ctl->vmax[i * 16 + j]);
-          }
-          exp_sync();
-          if (!failed) check(mbar_wait(&ctl->accfull, static_cast<uint32_t>(seg & 1), deadline, abort_flag));
-          if (!failed) {
-            tc_fence_after();
-            const __half* uh = reinterpret_cast<const __half*>(&ua);
-            const __half* uh2 = reinterpret_cast<const __half*>(&ub);
-            const float ginv = 1.0f / static_cast<float>(1 << (G - 1));
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-              int ch[16], cl[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) { ch[j] = 0; cl[j] = 0; }
-#pragma unroll
-              for (int g = 0; g < G; ++g) {
-                uint32_t vh[16], vl[16];
-                tmem_ld16(tmem + lane_base + g * NB + b * 16, vh);
-                tmem_ld16(tmem + lane_base + g * NB + 16 * B + b * 16, vl);
-                tc_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  ch[j] = 2 * ch[j] + static_cast<int>(vh[j]);
-                  cl[j] = 2 * cl[j] + static_cast<int>(vl[j]);
-                }
-              }
-              float acc = 0.0f;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float slo = ctl->sig_lo[b * 16 + j];
-                const float sbz = (256.0f * slo * static_cast<float>(ch[j]) + slo * static_cast<float>(cl[j])) * ginv;
-                // S = 1 - 2 Sb (bit 1 = sign -1):  T = sum_c Z - 2 sum_c Sb Z
-                const float tval = ctl->cseg[b * 16 + j] - 2.0f * sbz;
-                const float uj = __half2float(j < 8 ? uh[j] : uh2[j - 8]);
-                acc = fmaf(uj, tval, acc);
-              }
-              ypart[b] += acc;
-            }
-            tc_fence_before();
-            mbar_arrive(&ctl->accempty);
-          }
-          exp_sync();  // cseg and the scales are rewritten by the next segment
-          ++seg;
-        }
-
-        const bool rt_end = (u + 1 == u1) || (rem == per_rt - 1);
-        if (rt_end) {
-          const long long first_u = rt * per_rt, last_u = first_u + per_rt - 1;
-          const size_t row = static_cast<size_t>(rt) * kTileRows + tid;
-          if (first_u >= u0 && last_u < u1) {
-            if (!failed) {
-#pragma unroll
-              for (int b = 0; b < B; ++b) store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + row, ypart[b]);
-            }
-          } else {
-            const int slot2 = (rt == u0 / per_rt) ? 0 : 1;
-            float* mine = p.part + (static_cast<size_t>(cta) * 2 + slot2) * B * kTileRows;
-#pragma unroll
-            for (int b = 0; b < B; ++b) mine[b * kTileRows + tid] = ypart[b];
-            __threadfence();
-            exp_sync();
-            const int c_first = cta_of(first_u, U, grid), c_last = cta_of(last_u, U, grid);
-            if (tid == 0) {
-              unsigned long long* cp = p.cnt + rt;
-              unsigned long long expect = *reinterpret_cast<volatile unsigned long long*>(cp);
-              unsigned long long now = 0;
-              while (true) {
-                const bool same = static_cast<uint32_t>(expect >> 32) == tag;
-                const unsigned long long nv =
-                    same ? expect + 1ull : ((static_cast<unsigned long long>(tag) << 32) | 1ull);
-                const unsigned long long prev = atomicCAS(cp, expect, nv);
-                if (prev == expect) { now = nv; break; }
-                expect = prev;
-              }
-              ctl->is_last = static_cast<int>(now & 0xffffffffull) == (c_last - c_first + 1);
-            }
-            exp_sync();
-            if (ctl->is_last && !*abort_flag) {
-              __threadfence();
-              float acc[B];
-#pragma unroll
-              for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-              for (int c = c_first; c <= c_last; ++c) {
-                const long long cu0 = static_cast<long long>(c) * U / grid;
-                const int cslot = (rt == cu0 / per_rt) ? 0 : 1;
-                const float* pp = p.part + (static_cast<size_t>(c) * 2 + cslot) * B * kTileRows;
-#pragma unroll
-                for (int b = 0; b < B; ++b) acc[b] += __ldcg(pp + b * kTileRows + tid);
-              }
-#pragma unroll
-              for (int b = 0; b < B; ++b) store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + row, acc[b]);
-            }
-            exp_sync();  // is_last is rewritten by the next row tile
-          }
-#pragma unroll
-          for (int b = 0; b < B; ++b) ypart[b] = 0.0f;
+        if (++c == sg.len) {
+          // stage consumed (its words are in registers): release it to the copy warp
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->sempty[st]);
+          c = 0;
+          ++j;
+          if (j < nseg) sg = seg_of(s0 + j, p, C);
         }
       }
-      if (failed) set_error(p, ctl);
+      if (!failed) tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      named_sync(kBarA0 + half, 256);
+    }
+    if (failed) set_error(p, ctl);
+  } else if (warp < 8) {
+    // ------------------------------- activation chunks, epilogue, row tiles -------
+    const int tid = threadIdx.x - 128;   // row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
+    bool failed = false;
+    auto check = [&](bool ok) {
+      if (!__all_sync(0xffffffffu, ok)) failed = true;
+    };
+    // first chunk group: its inputs arrive by bulk copies
+    if (nseg > 0) {
+      check(mbar_wait(&ctl->vfull, 0, deadline, abort_flag) && mbar_wait(&ctl->xfull, 0, deadline, abort_flag));
+      produce_set<B>(sets, vscr, xscr, p.x_bf16, ctl, sg0, tid, &ctl->zfull[0], failed);
+    }
+    griddep_wait();   // the workspace and y belong to this launch only from here on
+    // chunk groups of this CTA: zk counts them; the set of group zk is zk & 1
+    int zk = 0;
+    int cur_cg = nseg > 0 ? sg0.cg : -1;
+    const int last_cg = nseg > 0 ? seg_of(s1 - 1, p, C).cg : -1;
+    if (nseg > 0 && last_cg > cur_cg) {   // second group: produce it now
+      const Seg sg2 = seg_of((cur_cg + 1) * p.RT, p, C);
+      load_set_inputs<B>(p, vscr, xscr, sg2, tid);
+      named_sync(kBarEpi, 128);
+      produce_set<B>(sets + K::SET, vscr, xscr, p.x_bf16, ctl, sg2, tid, &ctl->zfull[1], false);
+    }
+    const float ginv = 1.0f / static_cast<float>(1 << (G - 1));
+    for (int j = 0; j < nseg; ++j) {
+      const Seg sg = seg_of(s0 + j, p, C);
+      if (sg.cg != cur_cg) {
+        cur_cg = sg.cg;
+        ++zk;
+      }
+      const float* hdr = reinterpret_cast<const float*>(sets + (zk & 1) * K::SET);
+      const int acc = j & 1;
+      const int us = j % kURing;
+      // this row's U_i entries (16 fp16), from the U ring
+      if (!failed) check(mbar_wait(&ctl->ufull[us], static_cast<uint32_t>((j / kURing) & 1), deadline, abort_flag));
+      uint4 ua = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
+      if (!failed) {
+        ua = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32);
+        ub = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32 + 16);
+      }
+      if (!failed) check(mbar_wait(&ctl->accfull[acc], static_cast<uint32_t>((j >> 1) & 1), deadline, abort_flag));
+      if (!failed) {
+        tc_fence_after();
+        const __half* uh = reinterpret_cast<const __half*>(&ua);
+        const __half* uh2 = reinterpret_cast<const __half*>(&ub);
+        const uint32_t abase = tmem + lane_base + static_cast<uint32_t>(acc * G * NB);
+        float part[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          int ch[16], cl[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            ch[jj] = 0;
+            cl[jj] = 0;
+          }
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            uint32_t vh[16], vl[16];
+            tmem_ld16(abase + gg * NB + b * 16, vh);
+            tmem_ld16(abase + gg * NB + 16 * B + b * 16, vl);
+            tc_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              ch[jj] = 2 * ch[jj] + static_cast<int>(vh[jj]);
+              cl[jj] = 2 * cl[jj] + static_cast<int>(vl[jj]);
+            }
+          }
+          float sacc = 0.0f;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float slo = hdr[b * 16 + jj];
+            const float sbz = (256.0f * slo * static_cast<float>(ch[jj]) + slo * static_cast<float>(cl[jj])) * ginv;
+            // S = 1 - 2 Sb (bit 1 = sign -1):  T = sum_c Z - 2 sum_c Sb Z
+            const float tval = hdr[64 + b * 16 + jj] - 2.0f * sbz;
+            const float uj = __half2float(jj < 8 ? uh[jj] : uh2[jj - 8]);
+            sacc = fmaf(uj, tval, sacc);
+          }
+          part[b] = sacc;
+        }
+        float* dst = p.part + static_cast<size_t>(s0 + j) * B * kTileRows;
+#pragma unroll
+        for (int b = 0; b < B; ++b) dst[b * kTileRows + tid] = part[b];
+      }
+      // accumulator acc is read: hand it to the issuers for segment j + 2
+      tc_fence_before();
+      __syncwarp();
+      if (j + 2 < nseg) named_sync(kBarAcc0 + acc, 256);
+      // U slot us is read by every epilogue thread: refill it for segment j + kURing
+      named_sync(kBarEpi, 128);
+      if (tid == 0 && j + kURing < nseg) {
+        const Seg sn = seg_of(s0 + j + kURing, p, C);
+        mbar_arrive_expect_tx(&ctl->ufull[us], kTileBytes);
+        bulk_g2s(uring + us * kTileBytes, u_tile(p, sn.i, sn.rt), kTileBytes, &ctl->ufull[us]);
+      }
+      // The last segment of group zk is done: its MMAs have completed, so the set of
+      // zk can take group zk + 2 if this CTA has one.
+      const bool group_end = (j + 1 == nseg) || seg_of(s0 + j + 1, p, C).cg != cur_cg;
+      if (group_end && cur_cg + 2 <= last_cg) {
+        const Seg sg3 = seg_of((cur_cg + 2) * p.RT, p, C);
+        load_set_inputs<B>(p, vscr, xscr, sg3, tid);
+        named_sync(kBarEpi, 128);
+        produce_set<B>(sets + (zk & 1) * K::SET, vscr, xscr, p.x_bf16, ctl, sg3, tid, &ctl->zfull[zk & 1], false);
+      }
+    }
+    if (failed) set_error(p, ctl);
+
+    // ------------- row tiles: count the segments, then reduce the owned row tiles ---
+    // Row tile rt is reduced by CTA rt mod grid once all NC partials have arrived:
+    // fixed chunk-group order, so the sum is deterministic.
+    __threadfence();
+    named_sync(kBarEpi, 128);
+    if (tid == 0) ctl->abort_snap = *abort_flag;
+    named_sync(kBarEpi, 128);
+    if (!ctl->abort_snap) {
+      for (int e = tid; e < nseg; e += 128) atomicAdd(p.cnt + seg_of(s0 + e, p, C).rt, 1u);
+      const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
+      for (int rt = cta; rt < p.RT; rt += grid) {
+        if (tid == 0) {
+          bool ok = true;
+          while (ld_acquire_u32(p.cnt + rt) != static_cast<uint32_t>(NC)) {
+            if (*abort_flag || globaltimer_ns() > deadline) {
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+          ctl->red_ok = ok ? 1 : 0;
+          if (!ok) set_error(p, ctl);
+        }
+        named_sync(kBarEpi, 128);
+        if (ctl->red_ok) {
+          __threadfence();
+          const float* pp = p.part + static_cast<size_t>(rt) * B * kTileRows + tid;
+          constexpr int kBatch = 32 / B;   // loads in flight per thread
+          float acc[B];
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+          for (int c0 = 0; c0 < NC; c0 += kBatch) {
+            float v[kBatch][B];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+              for (int b = 0; b < B; ++b) v[u][b] = c0 + u < NC ? __ldcg(pp + (c0 + u) * stride + b * kTileRows) : 0.0f;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+              for (int b = 0; b < B; ++b) acc[b] += v[u][b];
+          }
+#pragma unroll
+          for (int b = 0; b < B; ++b)
+            store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + tid, acc[b]);
+          if (tid == 0) p.cnt[rt] = 0u;   // the next call starts from zero
+        }
+        named_sync(kBarEpi, 128);
+      }
+    }
+  } else if (warp < kWarpIss0 + 4) {
+    // ---------------------------------------------------------- MMA issuers -------
+    // All lanes of the four issuer warps walk the units and pass the named barriers;
+    // lane 0 of warp w < NI issues the MMAs of K-steps t with (t % G) % NI == w and
+    // commits once per A-buffer pair and once per segment.  These threads never wait
+    // on an mbarrier per unit: such a wait costs the issuing thread more than the
+    // MMAs it would issue.
+    const int w = warp - kWarpIss0;
+    const bool leader = lane == 0 && w < NI;
+    bool ok = true;
+    bool any = false;
+    int j = 0, c = 0, zk = -1, cur_cg = -1;
+    Seg sg = sg0;
+    uint32_t zbase = 0;
+    for (int g = 0; j < nseg; ++g) {
+      const int half = g & 1;
+      __syncwarp();
+      named_sync(kBarA0 + half, 256);
+      tc_fence_after();
+      for (int q = 0; q < kGroup && j < nseg; ++q) {
+        const int acc = j & 1;
+        if (c == 0) {   // segment j starts
+          __syncwarp();
+          if (j >= 2) named_sync(kBarAcc0 + acc, 256);
+          tc_fence_after();
+          if (sg.cg != cur_cg) {
+            cur_cg = sg.cg;
+            ++zk;
+            if (leader && ok)
+              ok = mbar_wait(&ctl->zfull[zk & 1], static_cast<uint32_t>((zk >> 1) & 1), deadline, abort_flag);
+            zbase = smem_u32(sets + (zk & 1) * K::SET + kSetHdr);
+          }
+        }
+        if (leader && ok) {
+          const uint32_t zaddr = zbase + static_cast<uint32_t>(c * K::ZB);
+          const uint32_t acol = kAcol0 + 64u * static_cast<uint32_t>(kGroup * half + q);
+          const uint32_t dcol = static_cast<uint32_t>(acc * G * NB);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int gg = t % G;
+            if (gg % NI != w) continue;
+            const uint64_t bdesc = smem_desc_noswizzle(zaddr + t * (NB / 8) * 256, 128, 256);
+            mma_i8_ts(tmem + dcol + gg * NB, tmem + acol + 8 * t, bdesc, IDESC, (c == 0 && t < G) ? 0u : 1u);
+          }
+          any = true;
+        }
+        if (++c == sg.len) {
+          if (leader && ok) tc_commit(&ctl->accfull[acc]);
+          c = 0;
+          ++j;
+          if (j < nseg) sg = seg_of(s0 + j, p, C);
+        }
+      }
+      if (leader && ok) tc_commit(&ctl->aempty[half]);
+    }
+    if (leader) {
+      if (!ok) set_error(p, ctl);
+      if (any) {
+        tc_commit(&ctl->drain[w]);
+        mbar_wait(&ctl->drain[w], 0, globaltimer_ns() + 100000000ull, nullptr);
+      }
+    }
+  } else if (warp == kWarpCopy && lane == 0) {
+    // ------------------------------------------------------ sign-tile copies -------
+    // x and 1/s of the first chunk group: only after the previous kernel in the
+    // stream has finished (it may have written them).
+    griddep_wait();
+    if (nseg > 0) {
+      const int cols = sg0.len * kTileCols, col0 = sg0.kgA * kTileCols;
+      const uint32_t xb = static_cast<uint32_t>(cols) * 2;
+      mbar_arrive_expect_tx(&ctl->xfull, xb * B + static_cast<uint32_t>(cols) * 4);
+      for (int b = 0; b < B; ++b)
+        bulk_g2s(xscr + b * K::COLS * 2, static_cast<const uint8_t*>(p.x) + (static_cast<size_t>(b) * p.d + col0) * 2, xb,
+                 &ctl->xfull);
+      bulk_g2s(xscr + K::COLS * B * 2, p.inv_s + col0, static_cast<uint32_t>(cols) * 4, &ctl->xfull);
+    }
+    for (; issued < nseg; ++issued) {
+      const int st = issued % NS;
+      if (!mbar_wait(&ctl->sempty[st], static_cast<uint32_t>((issued / NS - 1) & 1), deadline, abort_flag)) {
+        set_error(p, ctl);
+        break;
+      }
+      const Seg sg = seg_of(s0 + issued, p, C);
+      const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
+      mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
+      bulk_g2s(stages + st * K::STAGE,
+               p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
+                   (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
+               bytes, &ctl->sfull[st]);
+    }
+    // No copy may be in flight when the CTA exits: wait for the last use of every
+    // stage, the first-group inputs and the U ring (each bounded).
+    const uint64_t drain_by = globaltimer_ns() + 100000000ull;
+    for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q) {
+      if (p.inject_unreachable && q == 0) continue;
+      mbar_wait(&ctl->sfull[q % NS], static_cast<uint32_t>((q / NS) & 1), drain_by, nullptr);
+    }
+    if (nseg > 0) {
+      mbar_wait(&ctl->vfull, 0, drain_by, nullptr);
+      mbar_wait(&ctl->xfull, 0, drain_by, nullptr);
     }
   }
-  if (warp < 4) cp_async_wait<0>();   // no sign copy is in flight at exit
 
+  // U-ring copies are issued by epilogue thread 0 (and the set-up): drain them too.
+  if (warp == kWarpEpi0 && lane == 0) {
+    const uint64_t drain_by = globaltimer_ns() + 100000000ull;
+    for (int j = (nseg > kURing ? nseg - kURing : 0); j < nseg; ++j)
+      mbar_wait(&ctl->ufull[j % kURing], static_cast<uint32_t>((j / kURing) & 1), drain_by, nullptr);
+  }
+  tc_fence_before();
   __syncthreads();
-  if (warp == kWarpZ) {
+  if (warp == kWarpCopy) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
-  }
-  // The last CTA to leave advances the workspace epoch for the next launch.
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t done = atomicAdd(p.hdr + 1, 1u);
-    if (done == static_cast<uint32_t>(grid) - 1u) {
-      p.hdr[1] = 0u;
-      __threadfence();
-      atomicExch(p.hdr, ctl->epoch + 1u);
-    }
   }
 }
 
 template <int B>
 cudaError_t launch_b(const DecodeParams& p, int grid, cudaStream_t stream) {
-  // G groups of K-steps, limited by the 256 TMEM accumulator columns (G * 32B <= 256).
-  constexpr int G = (B == 1) ? 8 : (B == 2 ? 4 : 2);
-  auto kern = decode_kernel<B, G>;
-  const size_t smem = decode_smem_bytes(B, p.stages);
-  static int configured = 0;  // the attribute is set once (stream capture never sees it)
-  if (configured < static_cast<int>(smem)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  auto kern = decode_kernel<B>;
+  constexpr int smem = Cfg<B>::SMEM;
+  static bool configured[64] = {};   // the attribute is set once per device, outside any capture
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured = static_cast<int>(smem);
+    configured[dev] = true;
   }
-  kern<<<grid, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace
 
-size_t decode_smem_bytes(int batch, int /*stages*/) {
-  const int zs = zstages(batch);
-  return static_cast<size_t>(kSignAhead) * kTileBytes + static_cast<size_t>(zs) * zstage_bytes(batch) + kScratchBytes +
-         2 * zs * sizeof(uint64_t) + sizeof(Ctl) + 64;
+size_t decode_smem_bytes(int batch) {
+  switch (batch) {
+    case 1: return Cfg<1>::SMEM;
+    case 2: return Cfg<2>::SMEM;
+    case 3: return Cfg<3>::SMEM;
+    case 4: return Cfg<4>::SMEM;
+    default: return 0;
+  }
 }
 
-int decode_pick_stages(int /*batch*/) { return kSignAhead; }
-
-cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, int /*sm_count*/, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream) {
   switch (batch) {
     case 1: return launch_b<1>(p, grid, stream);
     case 2: return launch_b<2>(p, grid, stream);

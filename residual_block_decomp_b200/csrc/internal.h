@@ -15,27 +15,34 @@ constexpr int kTileRows = 128;         // rows of a sign tile / an MMA M tile
 constexpr int kTileCols = 256;         // columns of a sign tile / one decode unit
 constexpr int kTileBytes = 4096;       // bytes of one sign tile
 constexpr int kDecodeMaxBatch = 4;     // batches up to this run the factored decode kernel
-constexpr int kDecodeMaxBlocks = 64;   // loaded blocks the decode kernel stages |V| maxima for
-constexpr int kMaxGrid = 160;          // cap on the decode kernel's persistent grid
+constexpr int kDecodeMaxBlocks = 64;   // loaded blocks the decode path accepts
 constexpr uint32_t kErrTimeout = 1u;   // device error word bit: a bounded wait ran out
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Decode workspace carve-up (all regions 256-byte aligned).
+// Decode work unit: a segment = one 128-row tile x up to C consecutive 256-column
+// chunks of one block (C = decode_chunks_per_segment(batch)).  Segments are numbered
+// s = cg * RT + rt over chunk groups cg = i * NCB + (kg / C) of block i.
+__host__ __device__ constexpr int decode_chunks_per_segment(int batch) { return batch == 1 ? 4 : 2; }
+inline int decode_groups_per_block(int d, int batch) {
+  const int KG = d / kTileCols, C = decode_chunks_per_segment(batch);
+  return (KG + C - 1) / C;
+}
+
+// Decode workspace carve-up (256-byte aligned regions): one arrival counter per row
+// tile, then per-segment partial outputs.  The counters come first so that their
+// place does not move with n_loaded or batch: a workspace reused by calls with other
+// sizes still finds them at zero (every completed call leaves them at zero).
 struct DecodeWs {
-  size_t hdr, zq, csum, flags, part, cnt, total;
+  size_t cnt, part, total;
 };
 inline DecodeWs decode_ws_layout(int m, int d, int n, int batch) {
   DecodeWs w{};
-  const size_t KG = static_cast<size_t>(d) / kTileCols;
-  const size_t chunks = static_cast<size_t>(n) * KG;
+  const size_t RT = static_cast<size_t>(m) / kTileRows;
+  const size_t segs = RT * static_cast<size_t>(n) * decode_groups_per_block(d, batch);
   size_t off = 0;
-  w.hdr = off;   off = 256;  // {epoch, done}: see DecodeParams::hdr
-  w.zq = off;    off = align_up(off + chunks * 32u * batch * kTileCols, 256);
-  w.csum = off;  off = align_up(off + chunks * 16u * batch * sizeof(float), 256);
-  w.flags = off; off = align_up(off + chunks * sizeof(uint32_t), 256);
-  w.part = off;  off = align_up(off + static_cast<size_t>(kMaxGrid) * 2 * kTileRows * batch * sizeof(float), 256);
-  w.cnt = off;   off = align_up(off + static_cast<size_t>(m / kTileRows) * sizeof(unsigned long long), 256);
+  w.cnt = off;  off = align_up(off + RT * sizeof(uint32_t), 256);
+  w.part = off; off = align_up(off + segs * batch * kTileRows * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -46,21 +53,13 @@ struct DecodeParams {
   const void* x;               // batch x d, f16 or bf16
   void* y;                     // batch x m, same dtype
   const float* inv_s;          // d
-  const float* vmax;           // [capacity][16]: max_c |V_i[c, j]|
-  uint8_t* zq;                 // [n * KG] activation chunks, int8 planes, UMMA layout
-  float* csum;                 // [n * KG][16 * batch] column sums of the dequantised chunk
-  uint32_t* flags;             // [n * KG] chunk published at epoch
-  float* part;                 // [grid][2][batch][128] partial outputs
-  unsigned long long* cnt;     // [m / 128] epoch-tagged arrival counters
+  float* part;                 // [segs][batch][128] partial outputs of the segments
+  uint32_t* cnt;               // [RT] segments of the row tile reduced so far
   uint32_t* err;               // sticky device error word
-  uint32_t* hdr;               // workspace header {epoch, done}: a launch tags its flags and
-                               // counters with epoch + 1; the last CTA to exit advances epoch.
-                               // Zero before the workspace's first use.
-  int m, d, n, KG, RT;
-  long long units;             // RT * n * KG
-  int stages;                  // shared-memory ring depth
+  int m, d, n, KG, RT, NCB;    // NCB chunk groups per block
+  int segs;                    // RT * n * NCB
   int x_bf16;
-  int inject_unreachable;      // consumers wait for a tag no CTA publishes (timeout test)
+  int inject_unreachable;      // the first sign copy of every CTA is never issued (timeout test)
   unsigned long long timeout_ns;
 };
 
@@ -77,9 +76,8 @@ struct PrefillParams {
 
 // Launchers (decode.cu, prefill.cu, aux_kernels.cu).  They return cudaSuccess or the
 // launch error.
-cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, int sm_count, cudaStream_t stream);
-size_t decode_smem_bytes(int batch, int stages);
-int decode_pick_stages(int batch);
+cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream);
+size_t decode_smem_bytes(int batch);
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_u,
                            const CUtensorMap& tm_v, int bf16, cudaStream_t stream);
@@ -88,7 +86,6 @@ size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs);
 cudaError_t launch_reconstruct(const uint8_t* blocks, unsigned long long block_bytes, const float* inv_s, int m,
                                int d, int n, void* out, int dtype, cudaStream_t stream);
 cudaError_t launch_unpack(const uint8_t* record, int m, int d, int8_t* out, cudaStream_t stream);
-cudaError_t launch_vmax(const uint8_t* record, int m, int d, float* out16, cudaStream_t stream);
 
 }  // namespace bs
 
@@ -98,11 +95,11 @@ struct bs_stack_s {
   uint8_t* blocks;
   size_t block_bytes, dev_bytes;
   const float* inv_s;
-  float* vmax;
   uint32_t* err;
   int device, sm_count;
   unsigned long long timeout_ns;
   int inject_unreachable;
+  int scratch_dirty;       // an error was reported: bs_linear_no_alloc clears its scratch first
   CUtensorMap tm_u, tm_v;  // prefill operand maps over the whole block area
   int tmaps_ready;
 };

@@ -12,16 +12,18 @@
 // Host code may not use the array's name as a device address (on the host it is
 // only a stand-in symbol), so the first call on each device, with that device
 // current, asks the runtime for the array's device address with
-// cudaGetSymbolAddress, clears the array's first 256 bytes (the launch-epoch
-// header the decode kernel reads) and caches the address.  That first call is
-// synchronous; make it before any stream capture.  Nothing here calls cudaMalloc,
-// cudaFree or any other allocating routine.
+// cudaGetSymbolAddress, clears the whole array and caches the address.  That first
+// call is synchronous; make it before any stream capture.  Nothing here calls
+// cudaMalloc, cudaFree or any other allocating routine.
 //
 // All calls on a device share the one array, and it keeps whatever the previous call
-// left in it; the decode kernel tags its flags and counters with a per-launch epoch,
-// so no clearing is needed between calls.  Two calls whose kernels may overlap on the
-// GPU (different streams, no ordering between them) race on the array: order them on
-// one stream, or give them distinct workspaces through bs_linear.
+// left in it; a decode call that completes leaves its row-tile counters at zero, so
+// no clearing is needed between calls.  A call that ran out of a bounded wait may
+// leave counters behind: once bs_get_device_error has reported an error on a stack,
+// the next call here on that stack clears the array first (an asynchronous memset on
+// the call's stream).  Two calls whose kernels may overlap on the GPU (different
+// streams, no ordering between them) race on the array: order them on one stream,
+// or give them distinct workspaces through bs_linear.
 #include <mutex>
 
 #include "internal.h"
@@ -43,7 +45,7 @@ bs_status scratch_address(int device, void** out) {
   if (g_scratch_addr[device] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return BS_ERR_CUDA;
-    if (cudaMemset(p, 0, 256) != cudaSuccess) return BS_ERR_CUDA;
+    if (cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) return BS_ERR_CUDA;
     g_scratch_addr[device] = p;
   }
   *out = g_scratch_addr[device];
@@ -65,5 +67,9 @@ extern "C" bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int bat
   void* scratch = nullptr;
   const bs_status st = scratch_address(device, &scratch);
   if (st != BS_OK) return st;
+  if (stack->scratch_dirty) {
+    if (cudaMemsetAsync(scratch, 0, need, stream) != cudaSuccess) return BS_ERR_CUDA;
+    stack->scratch_dirty = 0;
+  }
   return bs_linear(stack, x, batch, dt, n_loaded, y, scratch, kStaticScratchBytes, stream);
 }

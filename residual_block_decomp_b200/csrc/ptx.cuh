@@ -19,6 +19,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialisation may start before the
+// kernel ahead of it in the stream has finished.  griddep_wait() blocks the calling
+// thread until that kernel has completed and its memory writes are visible;
+// griddep_launch_dependents() lets the next kernel in the stream start early.  Both
+// are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier ------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -79,7 +79,7 @@ class BitStackLinear:
         if need == 0:
             return None
         if self._ws is None or self._ws.numel() < need:
-            # zeroed once: the library keeps the workspace consistent from then on
+            # zeroed once: completed calls leave it consistent (device_error re-zeroes it)
             self._ws = torch.zeros(need, dtype=torch.uint8, device=self.device)
         return self._ws
 
@@ -112,7 +112,12 @@ class BitStackLinear:
         return self.dev_blocks[off:off + self.block_bytes]
 
     def device_error(self) -> int:
-        return B.bs_get_device_error(self.handle)
+        """Reads and clears the stack's sticky device error word.  After an error the
+        workspace's counters may be stale, so the layer's own workspace is zeroed."""
+        status = B.bs_get_device_error(self.handle)
+        if status != B.BS_OK and self._ws is not None:
+            self._ws.zero_()
+        return status
 
     def close(self) -> None:
         if self.handle:

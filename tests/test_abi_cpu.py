@@ -49,7 +49,8 @@ def test_device_and_workspace_sizes():
     assert R.bs_stack_device_bytes(100, 4096, 16, 8) == 0     # m % 128
     assert R.bs_stack_device_bytes(4096, 4096, 8, 8) == 0     # k != 16 on the GPU path
     ws = R.bs_workspace_bytes(4096, 4096, 16, 8, 1)
-    assert ws >= 8 * 4096 * 32      # the int8 activation planes alone
+    # one fp32 partial per 128-row tile x 4-chunk group x block and row, + row-tile counters
+    assert ws == 32 * (16 // 4) * 8 * 128 * 4 + 256
     assert R.bs_workspace_bytes(4096, 4096, 16, 8, 4) > ws
     assert R.bs_workspace_bytes(4096, 4096, 16, 0, 1) == 0    # n = 0 needs none
     assert R.bs_workspace_bytes(4096, 4096, 16, 8, 64) == 0   # prefill needs none

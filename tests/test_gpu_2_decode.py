@@ -81,3 +81,19 @@ def test_decode_shared_workspace_between_stacks():
     torch.cuda.synchronize()
     assert_close(ya, a.y_ref(x, 2), what="stack a")
     assert_close(yb, b.y_ref(x, 3), what="stack b")
+
+
+def test_decode_workspace_reused_across_n_and_batch():
+    """One workspace, sized for the largest call, serves calls with other n_loaded and
+    batch in any order: the row-tile counters sit at a fixed place and every call
+    leaves them at zero, while the partial outputs move with the sizes."""
+    st = cases.synthetic_stack(97, 512, 1024, 4, matrix=7)
+    layer = load_stack(st)
+    need = max(layer.workspace(n, b).numel() for n in (1, 4) for b in (1, 4))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for n, b in [(4, 1), (1, 1), (3, 4), (1, 2), (4, 4), (2, 1), (4, 1)]:
+        x, xt = cases.inputs(97, b, st.d, matrix=10 * n + b)
+        y = layer.forward(xt.cuda(), n, workspace=ws)
+        torch.cuda.synchronize()
+        assert layer.device_error() == 0
+        assert_close(y, st.y_ref(x, n), what=f"reused workspace n={n} b={b}")

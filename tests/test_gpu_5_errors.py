@@ -1,10 +1,10 @@
 """GPU: error paths of the C ABI, and the bounded-wait timeout path.
 
-The timeout is injected on the host: the decode call is told to wait for an
-activation-chunk flag value that no CTA ever publishes, with a 2 ms bound.  The
-kernel records BS_ERR_TIMEOUT in the stack's device error word, drains its copies,
-frees tensor memory and returns; the context stays usable, which the next call
-shows.  Nothing here faults, traps or hangs the GPU."""
+The timeout is injected on the host: the decode call is told to leave out the first
+sign-tile copy of every CTA, with a 2 ms bound on each wait.  The kernel records
+BS_ERR_TIMEOUT in the stack's device error word, drains its copies and MMAs, frees
+tensor memory and returns; the context stays usable, which the next call shows.
+Nothing here faults, traps or hangs the GPU."""
 import pytest
 import torch
 

@@ -6,10 +6,12 @@ bs_linear_no_alloc keeps its scratch in a fixed array inside the library.  This 
 calls it through the C ABI twice in a row and checks each output against the
 workspace entry point bs_linear on the same inputs, within the tolerance the other
 parity tests use.  It sits in a file of its own that pytest collects last."""
+import numpy as np
 import pytest
 import torch
 
 import residual_block_decomp_b200 as R
+from residual_block_decomp_b200 import BitStackLinear
 from tests import cases
 from tests.gpu_util import assert_close, load_stack
 
@@ -43,14 +45,7 @@ def test_no_alloc_rejects_oversize_and_prefill_batches():
     with pytest.raises(R.BsError) as e:
         R.bs_linear_no_alloc(layer.handle, x5, 5, y5)
     assert e.value.status == R.BS_ERR_INVALID_ARG
-    # 5 blocks of 128 x 16384 at batch 4 need more scratch than the 8 MiB array
-    assert R.bs_workspace_bytes(st.m, st.d, 16, 5, 4) > 8 << 20
-    x4 = torch.zeros((4, st.d), dtype=torch.float16, device="cuda")
-    y4 = torch.empty((4, st.m), dtype=torch.float16, device="cuda")
-    with pytest.raises(R.BsError) as e:
-        R.bs_linear_no_alloc(layer.handle, x4, 5, y4)
-    assert e.value.status == R.BS_ERR_CAPACITY
-    # the same stack at batch 1 fits, and agrees with the workspace entry point
+    # 128 x 16384, n = 5 at batch 1 fits, and agrees with the workspace entry point
     _, xt = cases.inputs(97, 1, st.d, matrix=7)
     x1 = xt.cuda()
     y_ws = layer.forward(x1, 5)
@@ -58,3 +53,17 @@ def test_no_alloc_rejects_oversize_and_prefill_batches():
     R.bs_linear_no_alloc(layer.handle, x1, 5, y1)
     torch.cuda.synchronize()
     assert_close(y1, y_ws.double().cpu().numpy(), what="128x16384 n=5 b=1")
+    # 9 blocks of 2048 x 16384 at batch 4 need more scratch than the 8 MiB array
+    # (zero records: only the size check runs)
+    m, d, n = 2048, 16384, 9
+    assert R.bs_workspace_bytes(m, d, 16, n, 4) > 8 << 20
+    big = BitStackLinear(m, d, n, np.ones(d, dtype=np.float32))
+    for _ in range(n):
+        big.add_record(np.zeros(big.block_bytes, dtype=np.uint8))
+    big.set_loaded(n)
+    torch.cuda.synchronize()
+    x4 = torch.zeros((4, d), dtype=torch.float16, device="cuda")
+    y4 = torch.empty((4, m), dtype=torch.float16, device="cuda")
+    with pytest.raises(R.BsError) as e:
+        R.bs_linear_no_alloc(big.handle, x4, n, y4)
+    assert e.value.status == R.BS_ERR_CAPACITY
