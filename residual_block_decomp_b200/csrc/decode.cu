@@ -51,24 +51,25 @@ constexpr int kThreads = 416;   // 13 warps
 constexpr int kWarpEpi0 = 4;    // warps 4..7: epilogue and activation-chunk production
 constexpr int kWarpIss0 = 8;    // warps 8..11: MMA issuers (lane 0 each)
 constexpr int kWarpCopy = 12;   // sign-tile copies; allocates TMEM
-constexpr int kABufs = 4;       // A-operand buffers in TMEM (64 columns each, from column 256): two pairs
-constexpr uint32_t kAcol0 = 256;
+constexpr int kNI = 4;          // MMA issuers: issuer w issues K-steps w and w + 4 of every unit
 constexpr int kMaxStages = 16;
+constexpr int kBarProd = 1;     // named barrier: warps 4-11 (the first chunk group)
 constexpr int kBarEpi = 2;      // named barrier: warps 4-7
-constexpr int kBarA0 = 3;       // named barriers 3, 4: expanders + issuers, A-buffer pair g & 1
-constexpr int kBarAcc0 = 5;     // named barriers 5, 6: epilogue + issuers, accumulator j & 1
 constexpr int kGroup = 2;       // units per A-buffer pair (the hand-over granularity)
-static_assert(2 * kGroup == kABufs, "two A-buffer pairs");
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kSetHdr = 512;    // per chunk-group set: sigma_lo[64], column sums[64]
 constexpr int kURing = 4;       // U tiles (4 KiB each) in flight ahead of the epilogue
+constexpr int kMaxPairs = 3;    // A-buffer pairs in tensor memory (one batch row: 3)
 
 struct Ctl {
   uint64_t sfull[kMaxStages], sempty[kMaxStages];
   uint64_t ufull[kURing];
-  uint64_t aempty[2];   // A-buffer pair free again: the MMAs that read it completed
+  uint64_t aempty[kMaxPairs];   // A-buffer pair free again: the MMAs that read it completed
   uint64_t accfull[2], zfull[2], drain[4];
   uint64_t vfull, xfull;  // inputs of the first chunk group: V rows; x rows and 1/s
+  uint32_t a_ready[4];    // A-buffer pairs stored, per expander warp (a sum could let a fast
+                          // warp stand in for a slow one)
+  uint32_t acc_free[2];   // accumulator zeroed by the epilogue: +1 per epilogue warp per release
   uint32_t tmem_base;
   int abort;
   int abort_snap;
@@ -81,23 +82,26 @@ template <int B>
 struct Cfg {
   static constexpr int NB = 32 * B;                 // MMA N: [hi plane 16B | lo plane 16B]
   static constexpr int ZB = NB * kTileCols;         // operand bytes of one chunk
-  static constexpr int G = B == 1 ? 4 : (B == 2 ? 2 : 1);
-  static constexpr int NI = G < 4 ? G : 4;          // issuer w owns groups g with g % NI == w
+  // Tensor memory: two accumulators of NB columns (double buffered across segments),
+  // then the A-buffer ring, 64 columns (128 lanes x 256 bytes) per unit, in pairs.
+  static constexpr uint32_t ACOL0 = 2 * NB;
+  static constexpr int NPAIRS = (512 - 2 * NB) / (64 * kGroup);
   static constexpr int C = decode_chunks_per_segment(B);
   static constexpr int COLS = C * kTileCols;        // columns of a chunk group
   static constexpr int SET = kSetHdr + C * ZB;      // one chunk-group set
   static constexpr int VSCR = COLS * kK * 2;        // V rows of a group (fp16)
   static constexpr int XSCR = COLS * B * 2 + COLS * 4;   // x rows (fp16/bf16), then 1/s (fp32)
+  static constexpr int XSF = COLS * B * 4;          // x (.) 1/s of the group (fp32)
   static constexpr int URING = kURing * kTileBytes; // U rows of a row tile (128 x 16 fp16) per slot
   static constexpr int STAGE = C * kTileBytes;
   static constexpr int CTL = static_cast<int>((sizeof(Ctl) + 127) / 128 * 128);
-  static constexpr int FIXED = 2 * SET + VSCR + XSCR + URING + CTL;
+  static constexpr int FIXED = 2 * SET + VSCR + XSCR + XSF + URING + CTL;
   static constexpr int NS0 = (kSmemLimit - FIXED) / STAGE;
   static constexpr int NS = NS0 < kMaxStages ? NS0 : kMaxStages;
   static constexpr int SMEM = NS * STAGE + FIXED;
   static_assert(NS >= 2, "sign ring too small");
-  static_assert(2 * G * NB <= static_cast<int>(kAcol0), "accumulators must fit below the A buffers");
-  static_assert(XSCR % 128 == 0 && VSCR % 128 == 0, "scratch alignment");
+  static_assert(NPAIRS >= 2 && NPAIRS <= kMaxPairs, "A-buffer ring");
+  static_assert(XSCR % 128 == 0 && VSCR % 128 == 0 && XSF % 128 == 0, "scratch alignment");
 };
 
 struct Seg {
@@ -161,18 +165,23 @@ __device__ void load_set_inputs(const DecodeParams& p, uint8_t* vscr, uint8_t* x
 
 // Quantises the activation chunks of chunk group `sg` (inputs already in the scratch:
 // V rows, x rows, 1/s) into `set`: operand planes in the UMMA no-swizzle K-major
-// layout, the per-column step sigma_lo and the dequantised column sum.  Run by the
-// 128 epilogue threads, which share named barrier kBarEpi; it has no other wait, so
-// every thread passes the same barriers.  `zfull` is signalled unless `skip`.
-template <int B>
-__device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xscr, int bf16, Ctl* ctl, const Seg& sg,
-                            int tid, uint64_t* zfull, bool skip) {
+// layout, the per-column step sigma_lo and the dequantised column sum.  Run by NT
+// threads that share named barrier `bar`; it has no other wait, so every thread passes
+// the same barriers.  `zfull` is signalled unless `skip`.
+template <int B, int NT>
+__device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xscr, float* xsf, int bf16, Ctl* ctl,
+                            const Seg& sg, int tid, int bar, uint64_t* zfull, bool skip) {
   using K = Cfg<B>;
-  constexpr int NT = 128;
   const int cols = sg.len * kTileCols;
   const __half* vh = reinterpret_cast<const __half*>(vscr);
   const uint16_t* xr = reinterpret_cast<const uint16_t*>(xscr);
   const float* isv = reinterpret_cast<const float*>(xscr + K::COLS * B * 2);
+  // x' = x (.) 1/s, once per column and batch row
+  for (int idx = tid; idx < B * cols; idx += NT) {
+    const int b = idx / cols, c = idx - b * cols;
+    xsf[b * K::COLS + c] = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
+  }
+  named_sync(bar, NT);
   const int items = (cols / 16) * 16 * B;   // (16-column group, column (b, j)), column fastest
   if (!skip) {
     // pass 1: max |Z| per column over the group; a thread folds its items of one
@@ -182,13 +191,11 @@ __device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xs
     for (int it = tid; it < items; it += NT) {
       const int c16 = it / (16 * B), col = it - c16 * 16 * B;
       const int b = col >> 4, j = col & 15;
+      const float* xp = xsf + b * K::COLS + c16 * 16;
+      const __half* vp = vh + c16 * 16 * kK + j;
       float mx = 0.0f;
 #pragma unroll
-      for (int kin = 0; kin < 16; ++kin) {
-        const int c = c16 * 16 + kin;
-        const float xs = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
-        mx = fmaxf(mx, fabsf(__fmul_rn(xs, __half2float(vh[c * kK + j]))));
-      }
+      for (int kin = 0; kin < 16; ++kin) mx = fmaxf(mx, fabsf(__fmul_rn(xp[kin], __half2float(vp[kin * kK]))));
       if (col != lcol) {
         if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
         lcol = col;
@@ -199,12 +206,12 @@ __device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xs
     }
     if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
   }
-  named_sync(kBarEpi, NT);
+  named_sync(bar, NT);
   if (!skip) {
     // pass 2: q = rint(Z / sigma_lo), |q| <= 127 * 256, q = 256 hi + lo
     uint8_t* ops = set + kSetHdr;
     int lcol = -1, lsum = 0;
-    float slo = 1.0f, rlo = 1.0f;
+    float rlo = 1.0f;
     for (int it = tid; it < items; it += NT) {
       const int c16 = it / (16 * B), col = it - c16 * 16 * B;
       const int b = col >> 4, j = col & 15;
@@ -213,15 +220,15 @@ __device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xs
         lcol = col;
         lsum = 0;
         const float amax = __int_as_float(ctl->amaxi[col]);
-        slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
+        const float slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
         rlo = 1.0f / slo;
       }
+      const float* xp = xsf + b * K::COLS + c16 * 16;
+      const __half* vp = vh + c16 * 16 * kK + j;
       uint32_t hw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int kin = 0; kin < 16; ++kin) {
-        const int c = c16 * 16 + kin;
-        const float xs = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
-        const float z = __fmul_rn(xs, __half2float(vh[c * kK + j]));
+        const float z = __fmul_rn(xp[kin], __half2float(vp[kin * kK]));
         int qv = __float2int_rn(z * rlo);
         qv = max(-32512, min(32512, qv));
         const int qh = (qv + 128) >> 8;
@@ -243,7 +250,7 @@ __device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xs
     if (lcol >= 0) atomicAdd(&ctl->zsum[lcol], lsum);
     fence_proxy_async_smem();   // the MMAs read the operands through the async proxy
   }
-  named_sync(kBarEpi, NT);
+  named_sync(bar, NT);
   if (tid < 16 * B) {
     if (!skip) {
       const float amax = __int_as_float(ctl->amaxi[tid]);
@@ -255,14 +262,14 @@ __device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xs
     ctl->amaxi[tid] = 0;
     ctl->zsum[tid] = 0;
   }
-  named_sync(kBarEpi, NT);
+  named_sync(bar, NT);
   if (tid == 0 && !skip) mbar_arrive(zfull);
 }
 
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
   using K = Cfg<B>;
-  constexpr int NB = K::NB, G = K::G, NI = K::NI, C = K::C, NS = K::NS;
+  constexpr int NB = K::NB, C = K::C, NS = K::NS, NPAIRS = K::NPAIRS;
   constexpr uint32_t IDESC = make_idesc(2u, 0u, 1u, 128u, NB);  // s32 <- u8 x s8, M=128, N=NB
 
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -270,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   uint8_t* sets = smem + NS * K::STAGE;
   uint8_t* vscr = sets + 2 * K::SET;
   uint8_t* xscr = vscr + K::VSCR;
-  uint8_t* uring = xscr + K::XSCR;
+  float* xsf = reinterpret_cast<float*>(xscr + K::XSCR);
+  uint8_t* uring = xscr + K::XSCR + K::XSF;
   Ctl* ctl = reinterpret_cast<Ctl*>(uring + K::URING);
   volatile int* abort_flag = &ctl->abort;
 
@@ -286,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   griddep_launch_dependents();
 
   // ------------------------------------------------------------------ set-up -----
-  int issued = 0;   // sign copies issued (copy warp, lane 0)
   if (warp == kWarpCopy) {
     tmem_alloc(&ctl->tmem_base, 512);
     if (lane == 0) {
@@ -295,43 +302,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         mbar_init(&ctl->sempty[s], 4);
       }
       for (int u = 0; u < kURing; ++u) mbar_init(&ctl->ufull[u], 1);
+      for (int q = 0; q < kMaxPairs; ++q) mbar_init(&ctl->aempty[q], kNI);
       for (int q = 0; q < 2; ++q) {
-        mbar_init(&ctl->aempty[q], NI);
-        mbar_init(&ctl->accfull[q], NI);
+        mbar_init(&ctl->accfull[q], kNI);
         mbar_init(&ctl->zfull[q], 1);
       }
       for (int w = 0; w < 4; ++w) mbar_init(&ctl->drain[w], 1);
       mbar_init(&ctl->vfull, 1);
       mbar_init(&ctl->xfull, 1);
       ctl->abort = 0;
+      for (int w = 0; w < 4; ++w) ctl->a_ready[w] = 0;
+      ctl->acc_free[0] = 0;
+      ctl->acc_free[1] = 0;
       for (int c = 0; c < 16 * kDecodeMaxBatch; ++c) {
         ctl->amaxi[c] = 0;
         ctl->zsum[c] = 0;
       }
       fence_barrier_init();
-      // Stack memory only, so these copies may start before the previous kernel in
-      // the stream has finished: V rows of the first chunk group, the first sign
-      // stages, the first U tiles.
-      if (nseg > 0) {
-        const uint32_t vb = static_cast<uint32_t>(sg0.len) * kTileCols * kK * 2;
-        mbar_arrive_expect_tx(&ctl->vfull, vb);
-        bulk_g2s(vscr, v_rows(p, sg0), vb, &ctl->vfull);
-      }
-      for (; issued < NS && issued < nseg; ++issued) {
-        if (p.inject_unreachable && issued == 0) continue;
-        const Seg sg = seg_of(s0 + issued, p, C);
-        const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
-        mbar_arrive_expect_tx(&ctl->sfull[issued], bytes);
-        bulk_g2s(stages + issued * K::STAGE,
-                 p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
-                     (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
-                 bytes, &ctl->sfull[issued]);
-      }
-      for (int j = 0; j < kURing && j < nseg; ++j) {
-        const Seg sg = seg_of(s0 + j, p, C);
-        mbar_arrive_expect_tx(&ctl->ufull[j], kTileBytes);
-        bulk_g2s(uring + j * kTileBytes, u_tile(p, sg.i, sg.rt), kTileBytes, &ctl->ufull[j]);
-      }
     }
   }
   tc_fence_before();
@@ -341,11 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 
   if (warp < 4) {
     // ------------------------------------------------ expanders (rows = lanes) -----
-    // Units are walked in order and handed to the issuers in pairs (A buffers
-    // 2 (g & 1) and 2 (g & 1) + 1) through named barrier kBarA0 + (g & 1), which the
-    // issuers also sync on, so neither side can run a generation ahead.  A thread
-    // whose wait ran out keeps walking in "failed" mode, skipping work but passing
-    // every named barrier; failure is decided per warp by vote.
+    // Units are walked in order and handed to the issuers in pairs (A-buffer pair
+    // g mod NPAIRS): warp w adds 1 to a_ready[w] (release) once its rows of the pair
+    // are in tensor memory; the issuers wait for all four.  A warp whose wait ran out stops signalling (the issuers'
+    // bounded waits then run out too); failure is decided per warp by vote.
     const int tid = threadIdx.x;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     bool failed = false;
@@ -354,32 +340,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     };
     int j = 0, c = 0;
     Seg sg = sg0;
-    for (int g = 0; j < nseg; ++g) {
-      const int half = g & 1;
-      if (!failed && g >= 2)
-        check(mbar_wait(&ctl->aempty[half], static_cast<uint32_t>(((g >> 1) - 1) & 1), deadline, abort_flag));
-      for (int q = 0; q < kGroup && j < nseg; ++q) {
+    for (int g = 0; j < nseg && !failed; ++g) {
+      const int pr = g % NPAIRS;
+      if (g >= NPAIRS)
+        check(mbar_wait(&ctl->aempty[pr], static_cast<uint32_t>((g / NPAIRS - 1) & 1), deadline, abort_flag));
+      for (int q = 0; q < kGroup && j < nseg && !failed; ++q) {
         const int st = j % NS;
-        if (c == 0 && !failed) check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
-        if (!failed) {
-          const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
-          const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
-          const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
-          const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-          const uint32_t abase = tmem + lane_base + kAcol0 + 64u * static_cast<uint32_t>(kGroup * half + q);
+        if (c == 0) check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
+        if (failed) break;
+        const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
+        const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
+        const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
+        const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        const uint32_t abase = tmem + lane_base + K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
+        // K-step t holds bit t of every byte of the unit's words: byte q of word pw is
+        // sign column 32 t + 4 pw + q (the device tile order), value 0 or 1
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t r[32];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
 #pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
-              const int t = 4 * h + tt;
-              const int gg = t % G;
-              const uint32_t mask = 0x01010101u << gg;
+          for (int tt = 0; tt < 4; ++tt) {
 #pragma unroll
-              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (t - gg)) & mask;
-            }
-            tmem_st32(abase + 32 * h, r);
+            for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (4 * h + tt)) & 0x01010101u;
           }
+          tmem_st32(abase + 32 * h, r);
         }
         if (++c == sg.len) {
           // stage consumed (its words are in registers): release it to the copy warp
@@ -390,225 +374,239 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (j < nseg) sg = seg_of(s0 + j, p, C);
         }
       }
-      if (!failed) tc_wait_st();
+      if (failed) break;
+      tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      named_sync(kBarA0 + half, 256);
+      if (lane == 0) red_release_shared_add(&ctl->a_ready[warp], 1u);
     }
     if (failed) set_error(p, ctl);
-  } else if (warp < 8) {
-    // ------------------------------- activation chunks, epilogue, row tiles -------
-    const int tid = threadIdx.x - 128;   // row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
-    bool failed = false;
-    auto check = [&](bool ok) {
-      if (!__all_sync(0xffffffffu, ok)) failed = true;
-    };
-    // first chunk group: its inputs arrive by bulk copies
+  } else if (warp < 12) {
+    // --------- warps 4-11: the first chunk group's activation chunks, together ------
+    const int tp = threadIdx.x - 128;   // 0..255
+    bool pfailed = false;
+    if (warp < 8) {
+      // accumulators start at zero (the MMAs only accumulate); release both
+      const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
+      uint32_t zr[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) zr[q] = 0u;
+#pragma unroll
+      for (int cc = 0; cc < 2 * NB; cc += 32) tmem_st32(tmem + lane_base + cc, zr);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        red_release_shared_add(&ctl->acc_free[0], 1u);
+        red_release_shared_add(&ctl->acc_free[1], 1u);
+      }
+    }
     if (nseg > 0) {
-      check(mbar_wait(&ctl->vfull, 0, deadline, abort_flag) && mbar_wait(&ctl->xfull, 0, deadline, abort_flag));
-      produce_set<B>(sets, vscr, xscr, p.x_bf16, ctl, sg0, tid, &ctl->zfull[0], failed);
+      const bool ok = mbar_wait(&ctl->vfull, 0, deadline, abort_flag) && mbar_wait(&ctl->xfull, 0, deadline, abort_flag);
+      pfailed = !__all_sync(0xffffffffu, ok);
+      // a warp that timed out still runs the set's barriers, skipping the work; the
+      // others see the abort flag it set
+      if (pfailed) set_error(p, ctl);
+      named_sync(kBarProd, 256);
+      produce_set<B, 256>(sets, vscr, xscr, xsf, p.x_bf16, ctl, sg0, tp, kBarProd, &ctl->zfull[0],
+                          *abort_flag != 0);
     }
-    griddep_wait();   // the workspace and y belong to this launch only from here on
-    // chunk groups of this CTA: zk counts them; the set of group zk is zk & 1
-    int zk = 0;
-    int cur_cg = nseg > 0 ? sg0.cg : -1;
-    const int last_cg = nseg > 0 ? seg_of(s1 - 1, p, C).cg : -1;
-    if (nseg > 0 && last_cg > cur_cg) {   // second group: produce it now
-      const Seg sg2 = seg_of((cur_cg + 1) * p.RT, p, C);
-      load_set_inputs<B>(p, vscr, xscr, sg2, tid);
-      named_sync(kBarEpi, 128);
-      produce_set<B>(sets + K::SET, vscr, xscr, p.x_bf16, ctl, sg2, tid, &ctl->zfull[1], false);
-    }
-    const float ginv = 1.0f / static_cast<float>(1 << (G - 1));
-    for (int j = 0; j < nseg; ++j) {
-      const Seg sg = seg_of(s0 + j, p, C);
-      if (sg.cg != cur_cg) {
-        cur_cg = sg.cg;
-        ++zk;
+    if (warp < 8) {
+      // ------------------------------- epilogue, later chunk groups, row tiles -----
+      const int tid = threadIdx.x - 128;   // row within the tile = TMEM lane
+      const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
+      bool failed = pfailed;
+      auto check = [&](bool ok) {
+        if (!__all_sync(0xffffffffu, ok)) failed = true;
+      };
+      griddep_wait();   // the workspace and y belong to this launch only from here on
+      // chunk groups of this CTA: zk counts them; the set of group zk is zk & 1
+      int zk = 0;
+      int cur_cg = nseg > 0 ? sg0.cg : -1;
+      const int last_cg = nseg > 0 ? seg_of(s1 - 1, p, C).cg : -1;
+      if (nseg > 0 && last_cg > cur_cg) {   // second group: produce it now
+        const Seg sg2 = seg_of((cur_cg + 1) * p.RT, p, C);
+        load_set_inputs<B>(p, vscr, xscr, sg2, tid);
+        named_sync(kBarEpi, 128);
+        produce_set<B, 128>(sets + K::SET, vscr, xscr, xsf, p.x_bf16, ctl, sg2, tid, kBarEpi, &ctl->zfull[1], false);
       }
-      const float* hdr = reinterpret_cast<const float*>(sets + (zk & 1) * K::SET);
-      const int acc = j & 1;
-      const int us = j % kURing;
-      // this row's U_i entries (16 fp16), from the U ring
-      if (!failed) check(mbar_wait(&ctl->ufull[us], static_cast<uint32_t>((j / kURing) & 1), deadline, abort_flag));
-      uint4 ua = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
-      if (!failed) {
-        ua = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32);
-        ub = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32 + 16);
-      }
-      if (!failed) check(mbar_wait(&ctl->accfull[acc], static_cast<uint32_t>((j >> 1) & 1), deadline, abort_flag));
-      if (!failed) {
-        tc_fence_after();
-        const __half* uh = reinterpret_cast<const __half*>(&ua);
-        const __half* uh2 = reinterpret_cast<const __half*>(&ub);
-        const uint32_t abase = tmem + lane_base + static_cast<uint32_t>(acc * G * NB);
-        float part[B];
+      uint32_t zr[32];
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-          int ch[16], cl[16];
+      for (int q = 0; q < 32; ++q) zr[q] = 0u;
+      for (int j = 0; j < nseg; ++j) {
+        const Seg sg = seg_of(s0 + j, p, C);
+        if (sg.cg != cur_cg) {
+          cur_cg = sg.cg;
+          ++zk;
+        }
+        const float* hdr = reinterpret_cast<const float*>(sets + (zk & 1) * K::SET);
+        const int acc = j & 1;
+        const int us = j % kURing;
+        // this row's U_i entries (16 fp16), from the U ring
+        if (!failed) check(mbar_wait(&ctl->ufull[us], static_cast<uint32_t>((j / kURing) & 1), deadline, abort_flag));
+        uint4 ua = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
+        if (!failed) {
+          ua = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32);
+          ub = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32 + 16);
+        }
+        if (!failed) check(mbar_wait(&ctl->accfull[acc], static_cast<uint32_t>((j >> 1) & 1), deadline, abort_flag));
+        if (!failed) {
+          tc_fence_after();
+          const __half* uh = reinterpret_cast<const __half*>(&ua);
+          const __half* uh2 = reinterpret_cast<const __half*>(&ub);
+          const uint32_t abase = tmem + lane_base + static_cast<uint32_t>(acc * NB);
+          float part[B];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            ch[jj] = 0;
-            cl[jj] = 0;
-          }
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
+          for (int b = 0; b < B; ++b) {
             uint32_t vh[16], vl[16];
-            tmem_ld16(abase + gg * NB + b * 16, vh);
-            tmem_ld16(abase + gg * NB + 16 * B + b * 16, vl);
+            tmem_ld16(abase + b * 16, vh);
+            tmem_ld16(abase + 16 * B + b * 16, vl);
             tc_wait_ld();
+            float sacc = 0.0f;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-              ch[jj] = 2 * ch[jj] + static_cast<int>(vh[jj]);
-              cl[jj] = 2 * cl[jj] + static_cast<int>(vl[jj]);
+              const float slo = hdr[b * 16 + jj];
+              const float sbz = 256.0f * slo * static_cast<float>(static_cast<int>(vh[jj])) +
+                                slo * static_cast<float>(static_cast<int>(vl[jj]));
+              // S = 1 - 2 Sb (bit 1 = sign -1):  T = sum_c Z - 2 sum_c Sb Z
+              const float tval = hdr[64 + b * 16 + jj] - 2.0f * sbz;
+              const float uj = __half2float(jj < 8 ? uh[jj] : uh2[jj - 8]);
+              sacc = fmaf(uj, tval, sacc);
             }
+            part[b] = sacc;
           }
-          float sacc = 0.0f;
+          // zero the accumulator for segment j + 2 and hand it back to the issuers
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float slo = hdr[b * 16 + jj];
-            const float sbz = (256.0f * slo * static_cast<float>(ch[jj]) + slo * static_cast<float>(cl[jj])) * ginv;
-            // S = 1 - 2 Sb (bit 1 = sign -1):  T = sum_c Z - 2 sum_c Sb Z
-            const float tval = hdr[64 + b * 16 + jj] - 2.0f * sbz;
-            const float uj = __half2float(jj < 8 ? uh[jj] : uh2[jj - 8]);
-            sacc = fmaf(uj, tval, sacc);
-          }
-          part[b] = sacc;
-        }
-        float* dst = p.part + static_cast<size_t>(s0 + j) * B * kTileRows;
-#pragma unroll
-        for (int b = 0; b < B; ++b) dst[b * kTileRows + tid] = part[b];
-      }
-      // accumulator acc is read: hand it to the issuers for segment j + 2
-      tc_fence_before();
-      __syncwarp();
-      if (j + 2 < nseg) named_sync(kBarAcc0 + acc, 256);
-      // U slot us is read by every epilogue thread: refill it for segment j + kURing
-      named_sync(kBarEpi, 128);
-      if (tid == 0 && j + kURing < nseg) {
-        const Seg sn = seg_of(s0 + j + kURing, p, C);
-        mbar_arrive_expect_tx(&ctl->ufull[us], kTileBytes);
-        bulk_g2s(uring + us * kTileBytes, u_tile(p, sn.i, sn.rt), kTileBytes, &ctl->ufull[us]);
-      }
-      // The last segment of group zk is done: its MMAs have completed, so the set of
-      // zk can take group zk + 2 if this CTA has one.
-      const bool group_end = (j + 1 == nseg) || seg_of(s0 + j + 1, p, C).cg != cur_cg;
-      if (group_end && cur_cg + 2 <= last_cg) {
-        const Seg sg3 = seg_of((cur_cg + 2) * p.RT, p, C);
-        load_set_inputs<B>(p, vscr, xscr, sg3, tid);
-        named_sync(kBarEpi, 128);
-        produce_set<B>(sets + (zk & 1) * K::SET, vscr, xscr, p.x_bf16, ctl, sg3, tid, &ctl->zfull[zk & 1], false);
-      }
-    }
-    if (failed) set_error(p, ctl);
-
-    // ------------- row tiles: count the segments, then reduce the owned row tiles ---
-    // Row tile rt is reduced by CTA rt mod grid once all NC partials have arrived:
-    // fixed chunk-group order, so the sum is deterministic.
-    __threadfence();
-    named_sync(kBarEpi, 128);
-    if (tid == 0) ctl->abort_snap = *abort_flag;
-    named_sync(kBarEpi, 128);
-    if (!ctl->abort_snap) {
-      for (int e = tid; e < nseg; e += 128) atomicAdd(p.cnt + seg_of(s0 + e, p, C).rt, 1u);
-      const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
-      for (int rt = cta; rt < p.RT; rt += grid) {
-        if (tid == 0) {
-          bool ok = true;
-          while (ld_acquire_u32(p.cnt + rt) != static_cast<uint32_t>(NC)) {
-            if (*abort_flag || globaltimer_ns() > deadline) {
-              ok = false;
-              break;
-            }
-            __nanosleep(64);
-          }
-          ctl->red_ok = ok ? 1 : 0;
-          if (!ok) set_error(p, ctl);
-        }
-        named_sync(kBarEpi, 128);
-        if (ctl->red_ok) {
-          __threadfence();
-          const float* pp = p.part + static_cast<size_t>(rt) * B * kTileRows + tid;
-          constexpr int kBatch = 32 / B;   // loads in flight per thread
-          float acc[B];
-#pragma unroll
-          for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-          for (int c0 = 0; c0 < NC; c0 += kBatch) {
-            float v[kBatch][B];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-              for (int b = 0; b < B; ++b) v[u][b] = c0 + u < NC ? __ldcg(pp + (c0 + u) * stride + b * kTileRows) : 0.0f;
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-              for (int b = 0; b < B; ++b) acc[b] += v[u][b];
-          }
-#pragma unroll
-          for (int b = 0; b < B; ++b)
-            store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + tid, acc[b]);
-          if (tid == 0) p.cnt[rt] = 0u;   // the next call starts from zero
-        }
-        named_sync(kBarEpi, 128);
-      }
-    }
-  } else if (warp < kWarpIss0 + 4) {
-    // ---------------------------------------------------------- MMA issuers -------
-    // All lanes of the four issuer warps walk the units and pass the named barriers;
-    // lane 0 of warp w < NI issues the MMAs of K-steps t with (t % G) % NI == w and
-    // commits once per A-buffer pair and once per segment.  These threads never wait
-    // on an mbarrier per unit: such a wait costs the issuing thread more than the
-    // MMAs it would issue.
-    const int w = warp - kWarpIss0;
-    const bool leader = lane == 0 && w < NI;
-    bool ok = true;
-    bool any = false;
-    int j = 0, c = 0, zk = -1, cur_cg = -1;
-    Seg sg = sg0;
-    uint32_t zbase = 0;
-    for (int g = 0; j < nseg; ++g) {
-      const int half = g & 1;
-      __syncwarp();
-      named_sync(kBarA0 + half, 256);
-      tc_fence_after();
-      for (int q = 0; q < kGroup && j < nseg; ++q) {
-        const int acc = j & 1;
-        if (c == 0) {   // segment j starts
+          for (int cc = 0; cc < NB; cc += 32) tmem_st32(abase + cc, zr);
+          tc_wait_st();
+          tc_fence_before();
           __syncwarp();
-          if (j >= 2) named_sync(kBarAcc0 + acc, 256);
-          tc_fence_after();
-          if (sg.cg != cur_cg) {
-            cur_cg = sg.cg;
-            ++zk;
-            if (leader && ok)
-              ok = mbar_wait(&ctl->zfull[zk & 1], static_cast<uint32_t>((zk >> 1) & 1), deadline, abort_flag);
-            zbase = smem_u32(sets + (zk & 1) * K::SET + kSetHdr);
-          }
-        }
-        if (leader && ok) {
-          const uint32_t zaddr = zbase + static_cast<uint32_t>(c * K::ZB);
-          const uint32_t acol = kAcol0 + 64u * static_cast<uint32_t>(kGroup * half + q);
-          const uint32_t dcol = static_cast<uint32_t>(acc * G * NB);
+          if (lane == 0) red_release_shared_add(&ctl->acc_free[acc], 1u);
+          float* dst = p.part + static_cast<size_t>(s0 + j) * B * kTileRows;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int gg = t % G;
-            if (gg % NI != w) continue;
+          for (int b = 0; b < B; ++b) dst[b * kTileRows + tid] = part[b];
+        }
+        // U slot us is read by every epilogue thread: refill it for segment j + kURing
+        named_sync(kBarEpi, 128);
+        if (tid == 0 && j + kURing < nseg) {
+          const Seg sn = seg_of(s0 + j + kURing, p, C);
+          mbar_arrive_expect_tx(&ctl->ufull[us], kTileBytes);
+          bulk_g2s(uring + us * kTileBytes, u_tile(p, sn.i, sn.rt), kTileBytes, &ctl->ufull[us]);
+        }
+        // The last segment of group zk is done: its MMAs have completed, so the set of
+        // zk can take group zk + 2 if this CTA has one.
+        const bool group_end = (j + 1 == nseg) || seg_of(s0 + j + 1, p, C).cg != cur_cg;
+        if (group_end && cur_cg + 2 <= last_cg) {
+          const Seg sg3 = seg_of((cur_cg + 2) * p.RT, p, C);
+          load_set_inputs<B>(p, vscr, xscr, sg3, tid);
+          named_sync(kBarEpi, 128);
+          produce_set<B, 128>(sets + (zk & 1) * K::SET, vscr, xscr, xsf, p.x_bf16, ctl, sg3, tid, kBarEpi,
+                              &ctl->zfull[zk & 1], false);
+        }
+      }
+      if (failed) set_error(p, ctl);
+
+      // ------------- row tiles: count the segments, then reduce the owned row tiles ---
+      // Row tile rt is reduced by CTA rt mod grid once all NC partials have arrived:
+      // fixed chunk-group order, so the sum is deterministic.
+      __threadfence();
+      named_sync(kBarEpi, 128);
+      if (tid == 0) ctl->abort_snap = *abort_flag;
+      named_sync(kBarEpi, 128);
+      if (!ctl->abort_snap) {
+        for (int e = tid; e < nseg; e += 128) atomicAdd(p.cnt + seg_of(s0 + e, p, C).rt, 1u);
+        const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
+        for (int rt = cta; rt < p.RT; rt += grid) {
+          if (tid == 0) {
+            bool ok = true;
+            while (ld_acquire_u32(p.cnt + rt) != static_cast<uint32_t>(NC)) {
+              if (*abort_flag || globaltimer_ns() > deadline) {
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+            ctl->red_ok = ok ? 1 : 0;
+            if (!ok) set_error(p, ctl);
+          }
+          named_sync(kBarEpi, 128);
+          if (ctl->red_ok) {
+            __threadfence();
+            const float* pp = p.part + static_cast<size_t>(rt) * B * kTileRows + tid;
+            constexpr int kBatch = 32 / B;   // loads in flight per thread
+            float acc[B];
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+            for (int c0 = 0; c0 < NC; c0 += kBatch) {
+              float v[kBatch][B];
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+                for (int b = 0; b < B; ++b)
+                  v[u][b] = c0 + u < NC ? __ldcg(pp + (c0 + u) * stride + b * kTileRows) : 0.0f;
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+                for (int b = 0; b < B; ++b) acc[b] += v[u][b];
+            }
+#pragma unroll
+            for (int b = 0; b < B; ++b)
+              store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + tid, acc[b]);
+            if (tid == 0) p.cnt[rt] = 0u;   // the next call starts from zero
+          }
+          named_sync(kBarEpi, 128);
+        }
+      }
+    } else if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuers -------
+      // Lane 0 of warp 8 + w issues K-steps w and w + 4 of every unit into the
+      // segment's accumulator (which the epilogue zeroes, so every MMA accumulates) and
+      // commits once per A-buffer pair and once per segment.  It waits for the
+      // expanders and the epilogue by polling shared counters: an mbarrier wait, or a
+      // whole warp walking the loop, costs the issuing thread more than its MMAs.
+      const int w = warp - kWarpIss0;
+      bool ok = !pfailed;
+      bool any = false;
+      int j = 0, c = 0, zk = -1, cur_cg = -1;
+      Seg sg = sg0;
+      uint32_t zbase = 0;
+      for (int g = 0; j < nseg && ok; ++g) {
+        const int pr = g % NPAIRS;
+        ok = poll_geq4(ctl->a_ready, static_cast<uint32_t>(g + 1), deadline, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        for (int q = 0; q < kGroup && j < nseg && ok; ++q) {
+          const int acc = j & 1;
+          if (c == 0) {   // segment j starts: its accumulator must be zeroed
+            ok = poll_geq(&ctl->acc_free[acc], 4u * static_cast<uint32_t>((j >> 1) + 1), deadline, abort_flag);
+            tc_fence_after();
+            if (sg.cg != cur_cg) {
+              cur_cg = sg.cg;
+              ++zk;
+              if (ok) ok = mbar_wait(&ctl->zfull[zk & 1], static_cast<uint32_t>((zk >> 1) & 1), deadline, abort_flag);
+              zbase = smem_u32(sets + (zk & 1) * K::SET + kSetHdr);
+            }
+            if (!ok) break;
+          }
+          const uint32_t zaddr = zbase + static_cast<uint32_t>(c * K::ZB);
+          const uint32_t acol = K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
+          const uint32_t dcol = static_cast<uint32_t>(acc * NB);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int t = w + kNI * h;
             const uint64_t bdesc = smem_desc_noswizzle(zaddr + t * (NB / 8) * 256, 128, 256);
-            mma_i8_ts(tmem + dcol + gg * NB, tmem + acol + 8 * t, bdesc, IDESC, (c == 0 && t < G) ? 0u : 1u);
+            mma_i8_ts(tmem + dcol, tmem + acol + 8 * t, bdesc, IDESC, 1u);
           }
           any = true;
+          if (++c == sg.len) {
+            tc_commit(&ctl->accfull[acc]);
+            c = 0;
+            ++j;
+            if (j < nseg) sg = seg_of(s0 + j, p, C);
+          }
         }
-        if (++c == sg.len) {
-          if (leader && ok) tc_commit(&ctl->accfull[acc]);
-          c = 0;
-          ++j;
-          if (j < nseg) sg = seg_of(s0 + j, p, C);
-        }
+        if (ok) tc_commit(&ctl->aempty[pr]);
       }
-      if (leader && ok) tc_commit(&ctl->aempty[half]);
-    }
-    if (leader) {
       if (!ok) set_error(p, ctl);
       if (any) {
         tc_commit(&ctl->drain[w]);
@@ -617,8 +615,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
   } else if (warp == kWarpCopy && lane == 0) {
     // ------------------------------------------------------ sign-tile copies -------
-    // x and 1/s of the first chunk group: only after the previous kernel in the
-    // stream has finished (it may have written them).
+    // Stack memory first (it may be read before the previous kernel in the stream has
+    // finished): V rows of the first chunk group, the first sign stages and U tiles;
+    // then x and 1/s of the first group, only after that kernel has finished.
+    int issued = 0;
+    if (nseg > 0) {
+      const uint32_t vb = static_cast<uint32_t>(sg0.len) * kTileCols * kK * 2;
+      mbar_arrive_expect_tx(&ctl->vfull, vb);
+      bulk_g2s(vscr, v_rows(p, sg0), vb, &ctl->vfull);
+    }
+    for (; issued < NS && issued < nseg; ++issued) {
+      if (p.inject_unreachable && issued == 0) continue;
+      const Seg sg = seg_of(s0 + issued, p, C);
+      const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
+      mbar_arrive_expect_tx(&ctl->sfull[issued], bytes);
+      bulk_g2s(stages + issued * K::STAGE,
+               p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
+                   (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
+               bytes, &ctl->sfull[issued]);
+    }
+    for (int j = 0; j < kURing && j < nseg; ++j) {
+      const Seg sg = seg_of(s0 + j, p, C);
+      mbar_arrive_expect_tx(&ctl->ufull[j], kTileBytes);
+      bulk_g2s(uring + j * kTileBytes, u_tile(p, sg.i, sg.rt), kTileBytes, &ctl->ufull[j]);
+    }
     griddep_wait();
     if (nseg > 0) {
       const int cols = sg0.len * kTileCols, col0 = sg0.kgA * kTileCols;
@@ -644,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                bytes, &ctl->sfull[st]);
     }
     // No copy may be in flight when the CTA exits: wait for the last use of every
-    // stage, the first-group inputs and the U ring (each bounded).
+    // stage and for the first-group inputs (each bounded).
     const uint64_t drain_by = globaltimer_ns() + 100000000ull;
     for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q) {
       if (p.inject_unreachable && q == 0) continue;
@@ -656,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
   }
 
-  // U-ring copies are issued by epilogue thread 0 (and the set-up): drain them too.
+  // U-ring copies are issued by epilogue thread 0 (and the copy thread): drain them too.
   if (warp == kWarpEpi0 && lane == 0) {
     const uint64_t drain_by = globaltimer_ns() + 100000000ull;
     for (int j = (nseg > kURing ? nseg - kURing : 0); j < nseg; ++j)

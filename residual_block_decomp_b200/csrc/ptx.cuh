@@ -39,14 +39,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// try_wait suspends the calling thread until the phase completes or a time limit
+// (the hint, in ns) passes, so a waiting warp does not take issue slots from the
+// warps that share its scheduler.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
       : "memory");
   return ok != 0;
 }
@@ -128,6 +131,37 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+// Shared-memory counters with CTA-scope release / acquire: the cheap hand-over between
+// warps of one CTA (an mbarrier wait costs the waiting thread far more).
+__device__ __forceinline__ uint32_t ld_acquire_shared_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_shared_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+// Waits until *ctr >= target, or until the deadline / abort flag.
+// Sleeps between polls so that the waiting warp leaves its scheduler to the others.
+__device__ __forceinline__ bool poll_geq(const uint32_t* ctr, uint32_t target, uint64_t deadline,
+                                         volatile int* abort_flag) {
+  while (ld_acquire_shared_u32(ctr) < target) {
+    if ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline) return false;
+    __nanosleep(20);
+  }
+  return true;
+}
+// Waits until all four counters ctr[0..3] are >= target.
+__device__ __forceinline__ bool poll_geq4(const uint32_t* ctr, uint32_t target, uint64_t deadline,
+                                          volatile int* abort_flag) {
+  while (true) {
+    const uint32_t a = ld_acquire_shared_u32(ctr), b = ld_acquire_shared_u32(ctr + 1);
+    const uint32_t c = ld_acquire_shared_u32(ctr + 2), d = ld_acquire_shared_u32(ctr + 3);
+    if (min(min(a, b), min(c, d)) >= target) return true;
+    if ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline) return false;
+    __nanosleep(20);
+  }
 }
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
