@@ -44,6 +44,23 @@ L2_FALLBACK = 126 * 2 ** 20
 
 
 # ------------------------------------------------------------------ helpers -------
+def max_over_ranks(values, device=None):
+    """Each value's maximum over all ranks (one all-reduce); unchanged for one rank.
+    Timing a multi-GPU job by its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_us_per_call(ms_total, steps, world):
+    """Whole-job figure: the (slowest rank's) time over the calls of all ranks."""
+    return ms_total * 1000.0 / (steps * world)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -272,12 +289,7 @@ def run_cuda(args, rank, world, local_rank):
 
     ms_e2e, _ = timed(run_e2e)
 
-    # max over ranks
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], device=dev)
 
     out = {
         "ms": ms, "ms_e2e": ms_e2e, "steps": args.steps, "e2e_steps": e2e_steps, "clocks": clocks,
@@ -430,7 +442,7 @@ def main():
 
     hbm, bf16, bf16_sus, src = peaks()
     us_step = res["ms"] * 1000.0 / args.steps                 # per call on one GPU
-    value = res["ms"] * 1000.0 / (args.steps * world)          # whole job: all calls of all ranks
+    value = job_us_per_call(res["ms"], args.steps, world)      # whole job: all calls of all ranks
     nbytes = res["bytes"]
     achieved = nbytes / (us_step * 1e-6) / 1e9                 # GB/s of the decode kernel
     i8_peak = bf16 * 2.0                                       # int8 dense = 2x bf16 (nominal ratio 4.5 / 2.25)
@@ -450,7 +462,7 @@ def main():
                      "bytes_per_launch": nbytes,
                      "tensor_i8_frac": round(2 * res["flops_factored"] * 1.0 / (us_step * 1e-6) / (i8_peak * 1e12), 4)},
         "cpu_baseline": cpu,
-        "e2e": {"value": round(res["ms_e2e"] * 1000.0 / (res["e2e_steps"] * world), 4), "unit": UNIT,
+        "e2e": {"value": round(job_us_per_call(res["ms_e2e"], res["e2e_steps"], world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": res["e2e_h2d"], "d2h_bytes_per_step": res["e2e_d2h"]},
         "gpu_launches": args.steps,
         "clocks": res["clocks"],

@@ -47,14 +47,15 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 416;   // 13 warps
-constexpr int kWarpEpi0 = 4;    // warps 4..7: epilogue and activation-chunk production
-constexpr int kWarpIss0 = 8;    // warps 8..11: MMA issuers (lane 0 each)
-constexpr int kWarpCopy = 12;   // sign-tile copies; allocates TMEM
+constexpr int kThreads = 544;   // 17 warps
+constexpr int kExpWarps = 8;    // warps 0..7: sign expanders, two teams of four (alternate unit pairs)
+constexpr int kWarpEpi0 = 8;    // warps 8..11: epilogue and activation-chunk production
+constexpr int kWarpIss0 = 12;   // warps 12..15: MMA issuers (lane 0 each)
+constexpr int kWarpCopy = 16;   // sign-tile copies; allocates TMEM
 constexpr int kNI = 4;          // MMA issuers: issuer w issues K-steps w and w + 4 of every unit
 constexpr int kMaxStages = 16;
-constexpr int kBarProd = 1;     // named barrier: warps 4-11 (the first chunk group)
-constexpr int kBarEpi = 2;      // named barrier: warps 4-7
+constexpr int kBarProd = 1;     // named barrier: warps 8-15 (the first chunk group)
+constexpr int kBarEpi = 2;      // named barrier: warps 8-11
 constexpr int kGroup = 2;       // units per A-buffer pair (the hand-over granularity)
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kSetHdr = 512;    // per chunk-group set: sigma_lo[64], column sums[64]
@@ -66,9 +67,9 @@ struct Ctl {
   uint64_t ufull[kURing];
   uint64_t aempty[kMaxPairs];   // A-buffer pair free again: the MMAs that read it completed
   uint64_t accfull[2], zfull[2], drain[4];
-  uint64_t vfull, xfull;  // inputs of the first chunk group: V rows; x rows and 1/s
-  uint32_t a_ready[4];    // A-buffer pairs stored, per expander warp (a sum could let a fast
-                          // warp stand in for a slow one)
+  uint64_t vfull;         // V rows of the first chunk group
+  uint32_t a_ready[kExpWarps];  // A-buffer pairs stored, per expander warp (a sum could let
+                                // a fast warp stand in for a slow one)
   uint32_t acc_free[2];   // accumulator zeroed by the epilogue: +1 per epilogue warp per release
   uint32_t tmem_base;
   int abort;
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (lane == 0) {
       for (int s = 0; s < kMaxStages; ++s) {
         mbar_init(&ctl->sfull[s], 1);
-        mbar_init(&ctl->sempty[s], 4);
+        mbar_init(&ctl->sempty[s], kExpWarps);
       }
       for (int u = 0; u < kURing; ++u) mbar_init(&ctl->ufull[u], 1);
       for (int q = 0; q < kMaxPairs; ++q) mbar_init(&ctl->aempty[q], kNI);
@@ -309,9 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       for (int w = 0; w < 4; ++w) mbar_init(&ctl->drain[w], 1);
       mbar_init(&ctl->vfull, 1);
-      mbar_init(&ctl->xfull, 1);
       ctl->abort = 0;
-      for (int w = 0; w < 4; ++w) ctl->a_ready[w] = 0;
+      for (int w = 0; w < kExpWarps; ++w) ctl->a_ready[w] = 0;
       ctl->acc_free[0] = 0;
       ctl->acc_free[1] = 0;
       for (int c = 0; c < 16 * kDecodeMaxBatch; ++c) {
@@ -326,47 +326,58 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp < 4) {
+  if (warp < kExpWarps) {
     // ------------------------------------------------ expanders (rows = lanes) -----
-    // Units are walked in order and handed to the issuers in pairs (A-buffer pair
-    // g mod NPAIRS): warp w adds 1 to a_ready[w] (release) once its rows of the pair
-    // are in tensor memory; the issuers wait for all four.  A warp whose wait ran out stops signalling (the issuers'
-    // bounded waits then run out too); failure is decided per warp by vote.
-    const int tid = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // Units are walked in order in pairs: pair g goes to A-buffer pair g mod NPAIRS and
+    // is expanded by team g & 1 (warps 0-3 or 4-7; warp % 4 is the TMEM lane quadrant).
+    // Every expander warp walks all units (so all agree on the sign stages, each of
+    // which all eight release) but expands only its team's pairs; warp e adds 1 to
+    // a_ready[e] (release) once its rows of a pair are in tensor memory, and the
+    // issuers wait for the four warps of the pair's team.  A warp whose wait ran out
+    // stops signalling (the issuers' bounded waits then run out too); failure is
+    // decided per warp by vote.
+    const int team = warp >> 2;
+    const int tid = (warp & 3) * 32 + lane;   // row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool failed = false;
     auto check = [&](bool ok) {
       if (!__all_sync(0xffffffffu, ok)) failed = true;
     };
-    int j = 0, c = 0;
+    int j = 0, c = 0, waited = -1;
     Seg sg = sg0;
     for (int g = 0; j < nseg && !failed; ++g) {
       const int pr = g % NPAIRS;
-      if (g >= NPAIRS)
+      const bool mine = (g & 1) == team;
+      if (mine && g >= NPAIRS)
         check(mbar_wait(&ctl->aempty[pr], static_cast<uint32_t>((g / NPAIRS - 1) & 1), deadline, abort_flag));
       for (int q = 0; q < kGroup && j < nseg && !failed; ++q) {
         const int st = j % NS;
-        if (c == 0) check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
-        if (failed) break;
-        const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
-        const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
-        const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
-        const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        const uint32_t abase = tmem + lane_base + K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
-        // K-step t holds bit t of every byte of the unit's words: byte q of word pw is
-        // sign column 32 t + 4 pw + q (the device tile order), value 0 or 1
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-#pragma unroll
-          for (int tt = 0; tt < 4; ++tt) {
-#pragma unroll
-            for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (4 * h + tt)) & 0x01010101u;
+        if (mine) {
+          if (waited != j) {
+            check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
+            waited = j;
           }
-          tmem_st32(abase + 32 * h, r);
+          if (failed) break;
+          const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
+          const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
+          const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
+          const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          const uint32_t abase = tmem + lane_base + K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
+          // K-step t holds bit t of every byte of the unit's words: byte q of word pw is
+          // sign column 32 t + 4 pw + q (the device tile order), value 0 or 1
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) {
+#pragma unroll
+              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (4 * h + tt)) & 0x01010101u;
+            }
+            tmem_st32(abase + 32 * h, r);
+          }
         }
         if (++c == sg.len) {
-          // stage consumed (its words are in registers): release it to the copy warp
+          // segment done (its words are in registers): release the stage to the copy warp
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->sempty[st]);
           c = 0;
@@ -375,17 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
       if (failed) break;
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) red_release_shared_add(&ctl->a_ready[warp], 1u);
+      if (mine) {
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) red_release_shared_add(&ctl->a_ready[warp], 1u);
+      }
     }
     if (failed) set_error(p, ctl);
-  } else if (warp < 12) {
-    // --------- warps 4-11: the first chunk group's activation chunks, together ------
-    const int tp = threadIdx.x - 128;   // 0..255
+  } else if (warp < kWarpIss0 + 4) {
+    // --------- warps 8-15: the first chunk group's activation chunks, together ------
+    const int tp = threadIdx.x - kWarpEpi0 * 32;   // 0..255
     bool pfailed = false;
-    if (warp < 8) {
+    if (warp < kWarpIss0) {
       // accumulators start at zero (the MMAs only accumulate); release both
       const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
       uint32_t zr[32];
@@ -402,7 +415,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
     }
     if (nseg > 0) {
-      const bool ok = mbar_wait(&ctl->vfull, 0, deadline, abort_flag) && mbar_wait(&ctl->xfull, 0, deadline, abort_flag);
+      // x and 1/s of the first group by plain loads (only after the previous kernel in
+      // the stream has finished: it may have written them), V rows by a bulk copy
+      griddep_wait();
+      {
+        const int cols = sg0.len * kTileCols, col0 = sg0.kgA * kTileCols;
+        uint16_t* xr = reinterpret_cast<uint16_t*>(xscr);
+        for (int idx = tp; idx < B * cols; idx += 256) {
+          const int b = idx / cols, c = idx - b * cols;
+          xr[b * K::COLS + c] = static_cast<const uint16_t*>(p.x)[static_cast<size_t>(b) * p.d + col0 + c];
+        }
+        float* isv = reinterpret_cast<float*>(xscr + K::COLS * B * 2);
+        for (int c = tp; c < cols; c += 256) isv[c] = __ldg(p.inv_s + col0 + c);
+      }
+      const bool ok = mbar_wait(&ctl->vfull, 0, deadline, abort_flag);
       pfailed = !__all_sync(0xffffffffu, ok);
       // a warp that timed out still runs the set's barriers, skipping the work; the
       // others see the abort flag it set
@@ -411,9 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       produce_set<B, 256>(sets, vscr, xscr, xsf, p.x_bf16, ctl, sg0, tp, kBarProd, &ctl->zfull[0],
                           *abort_flag != 0);
     }
-    if (warp < 8) {
+    if (warp < kWarpIss0) {
       // ------------------------------- epilogue, later chunk groups, row tiles -----
-      const int tid = threadIdx.x - 128;   // row within the tile = TMEM lane
+      const int tid = threadIdx.x - kWarpEpi0 * 32;   // row within the tile = TMEM lane
       const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
       bool failed = pfailed;
       auto check = [&](bool ok) {
@@ -572,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       uint32_t zbase = 0;
       for (int g = 0; j < nseg && ok; ++g) {
         const int pr = g % NPAIRS;
-        ok = poll_geq4(ctl->a_ready, static_cast<uint32_t>(g + 1), deadline, abort_flag);
+        ok = poll_geq4(ctl->a_ready + 4 * (g & 1), static_cast<uint32_t>((g >> 1) + 1), deadline, abort_flag);
         if (!ok) break;
         tc_fence_after();
         for (int q = 0; q < kGroup && j < nseg && ok; ++q) {
@@ -615,9 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
   } else if (warp == kWarpCopy && lane == 0) {
     // ------------------------------------------------------ sign-tile copies -------
-    // Stack memory first (it may be read before the previous kernel in the stream has
-    // finished): V rows of the first chunk group, the first sign stages and U tiles;
-    // then x and 1/s of the first group, only after that kernel has finished.
+    // Stack memory only (it may be read before the previous kernel in the stream has
+    // finished): V rows of the first chunk group, the first sign stages and U tiles.
     int issued = 0;
     if (nseg > 0) {
       const uint32_t vb = static_cast<uint32_t>(sg0.len) * kTileCols * kK * 2;
@@ -638,16 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const Seg sg = seg_of(s0 + j, p, C);
       mbar_arrive_expect_tx(&ctl->ufull[j], kTileBytes);
       bulk_g2s(uring + j * kTileBytes, u_tile(p, sg.i, sg.rt), kTileBytes, &ctl->ufull[j]);
-    }
-    griddep_wait();
-    if (nseg > 0) {
-      const int cols = sg0.len * kTileCols, col0 = sg0.kgA * kTileCols;
-      const uint32_t xb = static_cast<uint32_t>(cols) * 2;
-      mbar_arrive_expect_tx(&ctl->xfull, xb * B + static_cast<uint32_t>(cols) * 4);
-      for (int b = 0; b < B; ++b)
-        bulk_g2s(xscr + b * K::COLS * 2, static_cast<const uint8_t*>(p.x) + (static_cast<size_t>(b) * p.d + col0) * 2, xb,
-                 &ctl->xfull);
-      bulk_g2s(xscr + K::COLS * B * 2, p.inv_s + col0, static_cast<uint32_t>(cols) * 4, &ctl->xfull);
     }
     for (; issued < nseg; ++issued) {
       const int st = issued % NS;
@@ -670,10 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       if (p.inject_unreachable && q == 0) continue;
       mbar_wait(&ctl->sfull[q % NS], static_cast<uint32_t>((q / NS) & 1), drain_by, nullptr);
     }
-    if (nseg > 0) {
-      mbar_wait(&ctl->vfull, 0, drain_by, nullptr);
-      mbar_wait(&ctl->xfull, 0, drain_by, nullptr);
-    }
+    if (nseg > 0) mbar_wait(&ctl->vfull, 0, drain_by, nullptr);
   }
 
   // U-ring copies are issued by epilogue thread 0 (and the copy thread): drain them too.

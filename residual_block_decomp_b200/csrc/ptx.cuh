@@ -143,24 +143,23 @@ __device__ __forceinline__ void red_release_shared_add(uint32_t* p, uint32_t v) 
   asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 // Waits until *ctr >= target, or until the deadline / abort flag.
-// Sleeps between polls so that the waiting warp leaves its scheduler to the others.
+// Spins (a sleep between polls delayed the hand-over more than the spinning costs the
+// other warps); the deadline and abort flag are checked every 32 polls.
 __device__ __forceinline__ bool poll_geq(const uint32_t* ctr, uint32_t target, uint64_t deadline,
                                          volatile int* abort_flag) {
-  while (ld_acquire_shared_u32(ctr) < target) {
-    if ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline) return false;
-    __nanosleep(20);
+  for (uint32_t it = 1; ld_acquire_shared_u32(ctr) < target; ++it) {
+    if ((it & 31u) == 0u && ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline)) return false;
   }
   return true;
 }
-// Waits until all four counters ctr[0..3] are >= target.
+// Waits until all four counters ctr[0..3] are >= target (spinning, like poll_geq).
 __device__ __forceinline__ bool poll_geq4(const uint32_t* ctr, uint32_t target, uint64_t deadline,
                                           volatile int* abort_flag) {
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     const uint32_t a = ld_acquire_shared_u32(ctr), b = ld_acquire_shared_u32(ctr + 1);
     const uint32_t c = ld_acquire_shared_u32(ctr + 2), d = ld_acquire_shared_u32(ctr + 3);
     if (min(min(a, b), min(c, d)) >= target) return true;
-    if ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline) return false;
-    __nanosleep(20);
+    if ((it & 31u) == 0u && ((abort_flag != nullptr && *abort_flag) || globaltimer_ns() > deadline)) return false;
   }
 }
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
