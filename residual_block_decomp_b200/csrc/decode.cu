@@ -22,17 +22,21 @@
 //    (tcgen05.mma kind::i8) with exact int32 accumulation.  S = 1 - 2 Sb with Sb in
 //    {0, 1} the stored bit; the 1 part is the group's column sum, added in the epilogue.
 //  * Sign tiles (4 KiB per 128 x 256 unit, contiguous along a segment) stream from HBM
-//    by one 1-D bulk copy per segment into a ring of shared-memory stages, issued from
-//    the first instruction on.  Four warps expand sign bits in registers into u8
-//    operands (one AND, plus a shift when G < 8, per 4 columns: bytes {0, 2^g} for
-//    K-step t with g = t mod G; each g has its own TMEM accumulator and the epilogue
-//    recombines them exactly in int32) and store them to tensor memory (tcgen05.st).
-//    Up to four threads in four warps issue the MMAs; accumulators are double
-//    buffered so the epilogue of one segment overlaps the MMAs of the next.
-//  * The epilogue (four more warps) turns a segment's accumulators into one partial
-//    output per row and batch row.  When a CTA is done it counts its segments into
-//    per-row-tile counters; the CTA that completes a row tile sums its partials in
-//    fixed chunk-group order (deterministic) and resets the counter.
+//    by one 1-D bulk copy per segment into a ring of shared-memory stages.  Eight
+//    expander warps, two teams taking alternate unit pairs, turn each row's sign bits
+//    into u8 operands in registers (K-step t = bit t of every byte, one shift and one
+//    AND per 4 columns) and store them to a ring of A-buffer pairs in tensor memory
+//    (tcgen05.st).  Four threads in four warps issue the MMAs (K-steps w and w + 4 of
+//    every unit) into the segment's accumulator, which the epilogue zeroes after
+//    reading it, so every MMA accumulates; the two accumulators alternate between
+//    segments.  Expanders hand pairs to the issuers, and the epilogue hands
+//    accumulators back, through per-warp release counters in shared memory; MMA
+//    completion comes back through tcgen05.commit to mbarriers.
+//  * The epilogue (four more warps) turns a segment's accumulator into one partial
+//    output per row and batch row, with the row's U_i entries from a ring of U tiles.
+//    When a CTA is done it counts its segments into per-row-tile counters; CTA rt mod
+//    grid waits for all partials of row tile rt, sums them in fixed chunk-group order
+//    (deterministic), writes y and resets the counter.
 //  * The launch allows programmatic dependent launch: the prologue (barriers, TMEM,
 //    the first sign copies, V rows) runs before the previous kernel in the stream has
 //    finished; x, s, the workspace and y are touched only after griddepcontrol.wait.
