@@ -102,3 +102,28 @@ def test_reduction_reads_inside_workspace(m, d, n, b):
     # the last partial the reducer of the last row tile reads
     last = (RT - 1) * b * 128 + 127 + (NC - 1) * RT * b * 128 + (b - 1) * 128
     assert last < part_floats
+
+
+def test_expansion_rule_reads_columns_in_order():
+    """The decode expanders read, for row r of a tile, 16 bytes at r*16 and 16 at
+    2048 + r*16 (eight 32-bit words w[0..7]), and K-step t takes byte q of
+    (w[pw] >> t) & 0x01010101 as A[r, 32 t + 4 pw + q].  Applied to the library's own
+    host packer, that rule must give the signs in natural column order."""
+    import numpy as np
+    gen = np.random.default_rng(11)
+    m, d = 256, 512
+    neg = gen.random((m, d)) < 0.5
+    bits = np.packbits(neg, axis=1, bitorder="little")                  # canonical order
+    U = np.zeros((m, 16), np.float16)
+    V = np.zeros((d, 16), np.float16)
+    rec = R.bs_pack_record(m, d, 16, bits, U, V)
+    KG = d // 256
+    for rt in range(m // 128):
+        for kg in range(KG):
+            tile = rec[(rt * KG + kg) * 4096:(rt * KG + kg + 1) * 4096]
+            for r in range(128):
+                w = np.concatenate([tile[r * 16:r * 16 + 16], tile[2048 + r * 16:2048 + r * 16 + 16]]).view("<u4")
+                for t in range(8):
+                    a = ((w >> t) & 0x01010101).astype("<u4").view(np.uint8)   # bytes (pw, q)
+                    cols = kg * 256 + 32 * t + np.arange(32)
+                    assert np.array_equal(a.astype(bool), neg[rt * 128 + r, cols])
