@@ -207,6 +207,59 @@ def test_l1_record_roundtrip():
     assert np.array_equal(n2, neg) and np.array_equal(U2, U) and np.array_equal(V2, V)
 
 
+# ------------------------------------------------ activation scale (the reading) -----
+def test_activation_scale_is_per_channel_rms_with_floor():
+    """The stated reading of the scaling statistic (Review, Fig. 5 caption names
+    "Eq. 4" without printing it): s_c = sqrt(mean_r X[r, c]^2), floored at
+    1e-8 * max(s).  Hand-built columns whose RMS is known in closed form:
+      0: +-a alternating            -> a
+      1: a single spike b, else 0   -> b / sqrt(rows)
+      2: all zero                   -> the floor 1e-8 * max(s)
+      3: 3 and -4 alternating       -> sqrt((9 + 16) / 2)
+      4: constant c                 -> |c|
+    A mean of |X| (column 1 gives b / rows), a maximum of |X| (column 1 gives b,
+    column 3 gives 4), a missing floor (column 2 gives 0) or a missing square root
+    would each fail."""
+    rows = 64
+    a, b, c = 0.75, 12.0, -2.5
+    X = np.zeros((rows, 5))
+    X[:, 0] = np.where(np.arange(rows) % 2 == 0, a, -a)
+    X[17, 1] = b
+    X[:, 3] = np.where(np.arange(rows) % 2 == 0, 3.0, -4.0)
+    X[:, 4] = c
+    s = decompose.activation_scale(X)
+    expect = np.array([a, b / 8.0, 0.0, np.sqrt(12.5), abs(c)])
+    smax = expect.max()
+    expect[2] = 1e-8 * smax
+    assert np.allclose(s, expect, rtol=1e-15, atol=0.0)
+    # the scale is per input channel: permuting the columns permutes s
+    perm = np.array([3, 0, 4, 1, 2])
+    assert np.array_equal(decompose.activation_scale(X[:, perm]), s[perm])
+    # invariant to the order and sign of the calibration rows
+    assert np.allclose(decompose.activation_scale(-X[::-1]), s, rtol=1e-15, atol=0.0)
+
+
+def test_randomized_svd_reports_non_convergence(monkeypatch):
+    """The iteration never returns an unconverged result silently: with a tiny
+    singular gap and two iterations it reports converged=False, and strict mode
+    raises."""
+    gen = np.random.default_rng(5)
+    m, d, k = 120, 90, 4
+    Q1, _ = np.linalg.qr(gen.standard_normal((m, d)))
+    Q2, _ = np.linalg.qr(gen.standard_normal((d, d)))
+    sv = np.concatenate([[5.0, 4.0, 3.0, 2.0], 2.0 * (1.0 - 1e-3 * np.arange(1, d - k + 1) / d)])
+    A = (Q1 * np.sort(sv)[::-1]) @ Q2.T
+    monkeypatch.setattr(decompose, "EXACT_SVD_LIMIT", 10)
+    info = {}
+    decompose.truncated_svd(A, k, np.random.default_rng(0), max_iter=2, info=info)
+    assert info["method"] == "randomized" and info["iterations"] == 2 and info["converged"] is False
+    with pytest.raises(decompose.SvdNotConverged):
+        decompose.truncated_svd(A, k, np.random.default_rng(0), max_iter=2, strict=True)
+    info = {}
+    decompose.truncated_svd(A[:, :8], 4, None, info=info)     # LAPACK path
+    assert info == {"method": "lapack", "iterations": 0, "converged": True, "max_rel_change": 0.0}
+
+
 # ------------------------------------------------------------ randomized SVD --------
 def test_randomized_svd_matches_lapack_on_gapped_spectrum(monkeypatch):
     gen = np.random.default_rng(11)
@@ -216,7 +269,9 @@ def test_randomized_svd_matches_lapack_on_gapped_spectrum(monkeypatch):
     sv = np.concatenate([np.linspace(10, 5, k), 0.5 * np.exp(-np.arange(d - k) / 20)])
     A = (Q1 * sv) @ Q2.T
     monkeypatch.setattr(decompose, "EXACT_SVD_LIMIT", 10)
-    U, sig, Vt = decompose.truncated_svd(A, k, np.random.default_rng(0))
+    info = {}
+    U, sig, Vt = decompose.truncated_svd(A, k, np.random.default_rng(0), info=info, strict=True)
+    assert info["converged"] and info["method"] == "randomized"
     assert np.allclose(sig, sv[:k], rtol=1e-9)
     Ul, sl, Vtl = np.linalg.svd(A, full_matrices=False)
     assert np.allclose((U * sig) @ Vt, (Ul[:, :k] * sl[:k]) @ Vtl[:k], atol=1e-8)
@@ -255,6 +310,7 @@ def _pin_suite_passes():
         for case in [(7, 5, 2, 3, 2), (12, 9, 4, 4, 3)]:
             test_i5_forms_agree_with_brute_force(*case)
         test_i6_global_scale_factor_leaves_weight_unchanged()
+        test_activation_scale_is_per_channel_rms_with_floor()
     except AssertionError:
         return False
     return True
@@ -274,8 +330,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
     def dropped_block(negs, Us, Vs, n, m, d):
         return real_recon(negs, Us, Vs, max(n - 1, 0), m, d)
 
-    def flipped_sign(R, k, gen=None, round_fp16=True):
-        neg, U, V, Rn, sig = real_step(R, k, gen, round_fp16)
+    def flipped_sign(R, k, gen=None, round_fp16=True, info=None):
+        neg, U, V, Rn, sig = real_step(R, k, gen, round_fp16, info)
         S = np.where(neg, -1.0, 1.0)
         return ~neg, U, V, R + S * (U.astype(np.float64) @ V.astype(np.float64).T), sig
 
@@ -283,10 +339,16 @@ def test_planted_mistakes_are_caught(monkeypatch):
         y = real_fact(x, negs, Us, Vs, inv_s, n, m)
         return y * 1.0001
 
+    def mean_abs_scale(X):                            # mean |X| in place of the RMS
+        X = np.asarray(X, dtype=np.float64)
+        s = np.mean(np.abs(X), axis=0)
+        return np.maximum(s, 1e-8 * s.max())
+
     for name, mod, fn in [("reconstruct_scaled", linear, transposed_factor),
                           ("reconstruct_scaled", linear, dropped_block),
                           ("avd_step", decompose, flipped_sign),
-                          ("linear_factored", linear, scale_on_rows)]:
+                          ("linear_factored", linear, scale_on_rows),
+                          ("activation_scale", decompose, mean_abs_scale)]:
         with monkeypatch.context() as mp:
             mp.setattr(mod, name, fn)
             assert not _pin_suite_passes(), f"planted mistake in {name} ({fn.__name__}) went unnoticed"
