@@ -464,7 +464,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": round(job_us_per_call(res["ms_e2e"], res["e2e_steps"], world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": res["e2e_h2d"], "d2h_bytes_per_step": res["e2e_d2h"]},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps,       # one decode kernel per call
         "clocks": res["clocks"],
         "tokens_per_s": round(args.batch * 1e6 / value, 1),
         "weights_per_s": round(args.m * args.d * 1e6 / value, 1),

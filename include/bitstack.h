@@ -99,8 +99,10 @@ size_t bs_block_bytes(int m, int d, int k);
 size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks);
 
 /* Workspace bytes bs_linear needs for `n_loaded` blocks and `batch` rows (0 when the
- * call needs none): one partial output per (128-row tile, chunk group) and batch row,
- * and one arrival counter per row tile (about m * d * n * batch / 256 bytes).  The
+ * call needs none, i.e. n_loaded == 0 or batch > 4): one arrival counter per 128-row
+ * tile (first, so its place never moves), then one fp32 partial output per (128-row
+ * tile, chunk group of 4 x 256 columns at batch 1, else 2 x 256) and batch row, about
+ * m * d * n * batch / 256 bytes at batch 1 and m * d * n * batch / 128 above.  The
  * caller zeroes a workspace once before its first use (e.g. cudaMemsetAsync); every
  * call that completes leaves its counters at zero again, so no clearing is needed
  * between calls, and calls captured in a CUDA graph may be replayed.  After a call
@@ -137,35 +139,43 @@ bs_status bs_stack_destroy(bs_stack_t stack);
 /* Number of blocks currently held (loaded). */
 bs_status bs_stack_num_blocks(bs_stack_t stack, int* n_blocks);
 
-/* Loads the next block: one cudaMemcpyAsync of the record (ideally pinned host
- * memory, which must stay valid until the stream passes the copy) into slot
- * n_blocks, then a one-CTA kernel that stores max_c |V[c, j]| of the new block
- * (used to pick the int8 scale of the decode kernel's activations).  n_blocks += 1.
- * BS_ERR_CAPACITY when the stack is full. */
+/* Loads the next block when the memory budget grows: one cudaMemcpyAsync of the
+ * record (ideally pinned host memory, which must stay valid until the stream passes
+ * the copy) into slot n_blocks, with no repacking; n_blocks += 1.  BS_ERR_CAPACITY
+ * when the stack is full.  Source: review page, Fig. 2 caption (blocks are loaded
+ * from storage, in a presorted order, when the memory budget grows); OpenReview
+ * discussion, reply A1.B (the stack adapts to the available memory at run time). */
 bs_status bs_append_block(bs_stack_t stack, const void* host_record, bs_stream_t stream);
 
-/* Offloads the last block: n_blocks -= 1, no transfer (the host copy is the
- * storage).  BS_ERR_RANGE when the stack is empty. */
+/* Offloads the last block when the budget shrinks: n_blocks -= 1, no transfer (the
+ * host copy is the storage, and the blocks of one weight leave in the reverse order
+ * of their loading).  BS_ERR_RANGE when the stack is empty.  Source: review page,
+ * Fig. 2 caption (blocks are offloaded to storage when memory shrinks); OpenReview
+ * discussion, reply A1.B. */
 bs_status bs_drop_block(bs_stack_t stack);
 
 /* ----------------------------------------------------------------- compute ----- */
 
 /* y = x W_hat_n^T with n = n_loaded (0 <= n_loaded <= n_blocks; the decode path
  * takes up to 64 loaded blocks, the prefill path as many as its shared memory holds,
- * BS_ERR_RANGE / BS_ERR_CAPACITY beyond).
+ * BS_ERR_RANGE / BS_ERR_CAPACITY beyond).  W_hat_n is the sum over the first n
+ * blocks of sign (.) (U V^T), starting from zero, with the scaling undone per input
+ * channel: OpenReview discussion, weight restoration snippet; review page, Fig. 5
+ * caption ("Eq. 4").  The dense weight is never written to device memory.
  * x: batch x d row-major, y: batch x m row-major, both of dtype `dt` (BS_F16 or
  * BS_BF16), device pointers, 16-byte aligned.  n_loaded == 0 writes y = 0 (the
- * restoration accumulator starts at zero).  batch <= 4 runs the decode kernel (the
+ * restoration accumulator starts at zero).  batch <= 4 runs the decode path (the
  * factored form y = sum_i U_i (S_i ((x (.) 1/s) V_i)) with the +-1 contraction on
- * int8 tensor cores); larger batches run the prefill kernel (W_hat tiles rebuilt in
- * shared memory, then a tcgen05 GEMM).  workspace: >= bs_workspace_bytes(m, d, k,
+ * int8 tensor cores: a small kernel quantises the activations once per call, then
+ * the contraction kernel); larger batches run the prefill kernel (W_hat tiles rebuilt
+ * in shared memory, then a tcgen05 GEMM).  workspace: >= bs_workspace_bytes(m, d, k,
  * n_loaded, batch) device bytes, 256-aligned, zeroed before its first use (may be
  * NULL when the size is 0).  Asynchronous on `stream`; capturable in a CUDA graph.
- * The decode kernel is launched with programmatic dependent launch: it may start, and
- * read the stack's block area, before the kernel ahead of it on `stream` has
- * finished; it reads x and the scale vector and touches the workspace and y only
- * after that kernel has completed.  The block area is written only by this
- * library's own copies (bs_append_block), which a dependent launch never overtakes. */
+ * The decode kernels are launched with programmatic dependent launch: they may start,
+ * and read the stack's block area and the scale vector, before the kernel ahead of
+ * them on `stream` has finished; they read x and touch the workspace and y only after
+ * that kernel has completed.  The block area is written only by this library's own
+ * copies (bs_append_block), which a dependent launch never overtakes. */
 bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
                     void* workspace, size_t workspace_bytes, bs_stream_t stream);
 
@@ -175,20 +185,24 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
  * allocation after start-up (cudaMalloc may synchronise the device or fail under
  * memory pressure).  The pages have no counterpart to this call.
  * The scratch is an 8 MiB array inside the library, held by every GPU that loads
- * it until exit.  Calls whose scratch would exceed 8 MiB return BS_ERR_CAPACITY
- * (e.g. 4096 x 4096, n = 8 needs 0.5 MiB at batch 1); batch > 4 returns
+ * it until exit.  Calls whose scratch (bs_workspace_bytes) would exceed 8 MiB return
+ * BS_ERR_CAPACITY (e.g. 4096 x 4096 needs 0.5 MiB at n = 8, batch 1, and fits up to
+ * n = 64 at batch 1, 32 at batch 2, 21 at batch 3, 16 at batch 4); batch > 4 returns
  * BS_ERR_INVALID_ARG; the current device must be the stack's (BS_ERR_INVALID_ARG).
  * The first call on each device looks up the array's device address synchronously,
- * so make it before any stream capture; after bs_get_device_error has reported an
- * error on a stack, the next call on that stack clears the array first.  All calls on a device
- * share the array: calls that can overlap on the GPU race; order them on one
- * stream.  Allocates nothing.  Otherwise as bs_linear. */
+ * so make it before any stream capture.  All calls on a device, whatever their stack,
+ * share the array: once bs_get_device_error has reported an error on any stack of a
+ * device, the next call here on that device clears the whole array first.  Calls that
+ * can overlap on the GPU race on the array; order them on one stream.  Allocates
+ * nothing.  Otherwise as bs_linear. */
 bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
                              bs_stream_t stream);
 
 /* W_out = W_hat_n (m x d row-major, dtype BS_F32, BS_F16 or BS_BF16), for tests and
- * for users who want the dense weight (the unfused path of the restoration
- * snippet).  Asynchronous on `stream`. */
+ * for users who want the dense weight: the unfused path of the OpenReview
+ * discussion's weight restoration snippet (a zero accumulator, then unpack(sign)
+ * (.) (U V^T) added per loaded block), with the scaling undone per input channel
+ * (review page, Fig. 5 caption).  n == 0 writes zeros.  Asynchronous on `stream`. */
 bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_stream_t stream);
 
 /* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
@@ -206,9 +220,9 @@ const char* bs_status_string(bs_status status);
 /* Sets the bound (nanoseconds) on every device-side wait of this stack's kernels
  * (default 500 ms; values < 1000 are raised to 1000).  With `unreachable_flag`
  * non-zero, the next bs_linear decode call leaves out the first sign-tile copy of
- * every CTA, so the waits for it (and everything behind them) run out: a host-side
- * way to exercise the timeout path without faulting the GPU.  Zero the workspace
- * before reusing it after that call. */
+ * its first CTA, so that CTA's waits for it (and everything behind them) run out
+ * while the other CTAs complete: a host-side way to exercise the timeout path
+ * without faulting the GPU.  Zero the workspace before reusing it after that call. */
 bs_status bs_debug_set_wait(bs_stack_t stack, long long timeout_ns, int unreachable_flag);
 
 #ifdef __cplusplus

@@ -228,7 +228,12 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
     p.inject_unreachable = stack->inject_unreachable;
     stack->inject_unreachable = 0;
     p.timeout_ns = stack->timeout_ns;
-    const int grid = segs < stack->sm_count ? static_cast<int>(segs) : stack->sm_count;
+    // One CTA per SM, with a few SMs left over: calls chained on a stream start while the
+    // CTAs of the call ahead that add its last partials still reduce and write y, so the
+    // next call's CTAs find free SMs at once instead of queueing behind them.
+    const int slack = stack->sm_count > 32 ? 4 : 0;
+    const int ctas = stack->sm_count - slack;
+    const int grid = segs < ctas ? static_cast<int>(segs) : ctas;
     return cuda_status(launch_decode(p, batch, grid, stream));
   }
 
@@ -286,7 +291,7 @@ bs_status bs_get_device_error(bs_stack_t stack) {
   uint32_t v = 0;
   if (cudaMemcpy(&v, stack->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BS_ERR_CUDA;
   if (v == 0) return BS_OK;
-  stack->scratch_dirty = 1;
+  bs::note_device_error(stack->device);
   if (cudaMemset(stack->err, 0, sizeof(v)) != cudaSuccess) return BS_ERR_CUDA;
   return (v & kErrTimeout) ? BS_ERR_TIMEOUT : BS_ERR_CUDA;
 }

@@ -1,5 +1,4 @@
-// Auxiliary kernels: dense reconstruction of W_hat, sign unpacking, and the per-block
-// column maxima of |V| that the decode kernel's activation scales use.
+// Auxiliary kernels: dense reconstruction of W_hat and sign unpacking.
 //
 // Reconstruction follows the weight restoration snippet of the OpenReview discussion
 // of "BitStack: Any-Size Compression of Large Language Models in Variable Memory

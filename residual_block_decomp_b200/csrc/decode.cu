@@ -1,45 +1,52 @@
-// Decode kernel of the BitStack linear: y = sum_i U_i (S_i ((x (.) 1/s) (.) V_i)).
+// Decode path of the BitStack linear (a few rows of x):
+//     y = sum_i U_i (S_i ((x (.) 1/s) (.) V_i)).
 //
-// The weight of a BitStack layer is the sum of the loaded residual blocks, each a
-// +-1 sign matrix times the rank-k product of its singular vectors, with the
+// The weight of a BitStack layer is the sum of the loaded residual blocks, each a +-1
+// sign matrix times the rank-k product of its singular vectors, with the
 // activation-aware scale undone per input channel (weight restoration snippet of the
 // OpenReview discussion of "BitStack: Any-Size Compression of Large Language Models in
 // Variable Memory Environments"; review page "BitStack: Fine-Grained Size Control...",
-// Figs. 3 and 5).  For a few rows of x the kernel never forms that weight: by
-// associativity  y[b, r] = sum_i sum_j U_i[r, j] T_i[r, (j, b)],
-// T_i = S_i Z_i,  Z_i[c, (j, b)] = x[b, c] / s_c * V_i[c, j],  a +-1 contraction with
-// N = 16 * batch columns per block.
+// Figs. 3 and 5).  For a few rows of x the weight is never formed: by associativity
+//     y[b, r] = sum_i sum_j U_i[r, j] T_i[r, (b, j)],   T_i = S_i Z_i,
+//     Z_i[c, (b, j)] = x[b, c] / s_c * V_i[c, j],
+// a +-1 contraction with 16 * batch columns per block.
 //
-// How it maps to sm_100a:
-//  * Work is cut into segments: one 128-row tile of one block times C consecutive
-//    256-column chunks (C = 4 for one row of x, 2 for more).  Segments are numbered
-//    chunk-group-major (s = cg * RT + rt) and every CTA of the persistent grid takes
-//    a contiguous run of them, so a CTA touches one or two chunk groups.
-//  * Each CTA quantises the activation chunks of its own chunk groups (no exchange
-//    between CTAs): Z = (x / s) (.) V for the group's columns, per column (b, j) a
-//    step sigma = max |Z| / 32512 over the group, q = rint(Z / sigma) split exactly
-//    into two int8 planes q = 256 hi + lo.  So S_i Z_i runs on the int8 tensor cores
-//    (tcgen05.mma kind::i8) with exact int32 accumulation.  S = 1 - 2 Sb with Sb in
-//    {0, 1} the stored bit; the 1 part is the group's column sum, added in the epilogue.
-//  * Sign tiles (4 KiB per 128 x 256 unit, contiguous along a segment) stream from HBM
-//    by one 1-D bulk copy per segment into a ring of shared-memory stages.  Eight
-//    expander warps, two teams taking alternate unit pairs, turn each row's sign bits
-//    into u8 operands in registers (K-step t = bit t of every byte, one shift and one
-//    AND per 4 columns) and store them to a ring of A-buffer pairs in tensor memory
-//    (tcgen05.st).  Four threads in four warps issue the MMAs (K-steps w and w + 4 of
-//    every unit) into the segment's accumulator, which the epilogue zeroes after
-//    reading it, so every MMA accumulates; the two accumulators alternate between
-//    segments.  Expanders hand pairs to the issuers, and the epilogue hands
-//    accumulators back, through per-warp release counters in shared memory; MMA
-//    completion comes back through tcgen05.commit to mbarriers.
-//  * The epilogue (four more warps) turns a segment's accumulator into one partial
-//    output per row and batch row, with the row's U_i entries from a ring of U tiles.
-//    When a CTA is done it counts its segments into per-row-tile counters; CTA rt mod
-//    grid waits for all partials of row tile rt, sums them in fixed chunk-group order
-//    (deterministic), writes y and resets the counter.
-//  * The launch allows programmatic dependent launch: the prologue (barriers, TMEM,
-//    the first sign copies, V rows) runs before the previous kernel in the stream has
-//    finished; x, s, the workspace and y are touched only after griddepcontrol.wait.
+// One persistent launch, one CTA per SM, walking a contiguous run of segments (one
+// 128-row tile x one chunk group of C 256-column chunks of one block), numbered
+// chunk-group-major; with no more chunk groups than CTAs, each CTA's run lies inside
+// one chunk group:
+//  * Activation sets.  Z of a chunk group is quantised per column (b, j): a step
+//    sigma = max |Z| / 32512 over the group, q = rint(Z / sigma) split exactly into two
+//    int8 planes q = 256 hi + lo, written to shared memory in the tensor-core operand
+//    layout, with sigma and the integer column sums of q kept aside.  The CTA's first
+//    group is built by all its warps at the start from shared-memory copies of its V
+//    rows, 1/s and x (bulk-copied by the copy thread; V and 1/s before the kernel ahead
+//    has finished); maxima and sums are warp reduce-scatters; its second group by the epilogue
+//    warps while the first is being contracted, and later groups by the epilogue warps
+//    into the slot a finished group frees.
+//  * Signs.  A copy thread streams each segment's sign tiles (C x 4 KiB, contiguous in
+//    the record) into a ring of shared-memory stages with 1-D bulk copies, starting
+//    before the kernel ahead in the stream has finished (it reads only the block area).
+//  * Expansion.  T teams of four warps (one warp per tensor-memory lane quadrant) take
+//    the units (128 x 256 signs) in turn: each thread turns its row's 256 sign bits into
+//    s8 operands -128 Sb (K-step t = bit t of every byte moved to bit 7 by a multiply,
+//    which runs on the FMA pipe, then one AND per four columns; the device tile order)
+//    and stores them to one of its team's two slots in tensor memory; each warp then
+//    arrives on the slot's mbarrier.  No barrier inside a team.
+//  * MMA.  kNI issuer warps take the units in turn (warp-uniform, one elected lane
+//    issues): the unit's eight tcgen05.mma.kind::i8 (M = 128, N = 32 * batch, K = 32,
+//    s32 accumulate) into the segment's accumulator, then one commit that frees the slot
+//    and one that counts the unit into the segment's accumulator barrier.
+//  * Epilogue.  S = 1 - 2 Sb with Sb the stored bit, so T = colsum(Z) - 2 Sb Z; four
+//    warps read a finished accumulator (hi and lo planes), form T with the group's sigma
+//    and column sums, apply the row's U_i entries and store one fp32 partial per row and
+//    batch row; they zero the accumulator for reuse (every MMA accumulates; int32 sums
+//    are exact, so the order of the units does not matter).
+//  * Reduction.  At the end every CTA counts its partials into per-row-tile arrival
+//    counters; the CTA that adds a tile's last partial sums all of them in fixed
+//    chunk-group order and writes y: deterministic, and no CTA ever waits for another.
+//  * Hand-overs between roles are mbarriers, waited on with the suspending try_wait so
+//    that a waiting warp takes no issue slots from the warps that expand signs.
 //  * Every wait is bounded; a wait that runs out sets the device error word, and the
 //    CTA drains its copies and MMAs, frees tensor memory and returns.
 #include <cuda_bf16.h>
@@ -51,277 +58,420 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 544;   // 17 warps
-constexpr int kExpWarps = 8;    // warps 0..7: sign expanders, two teams of four (alternate unit pairs)
-constexpr int kWarpEpi0 = 8;    // warps 8..11: epilogue and activation-chunk production
-constexpr int kWarpIss0 = 12;   // warps 12..15: MMA issuers (lane 0 each)
-constexpr int kWarpCopy = 16;   // sign-tile copies; allocates TMEM
-constexpr int kNI = 4;          // MMA issuers: issuer w issues K-steps w and w + 4 of every unit
 constexpr int kMaxStages = 16;
-constexpr int kBarProd = 1;     // named barrier: warps 8-15 (the first chunk group)
-constexpr int kBarEpi = 2;      // named barrier: warps 8-11
-constexpr int kGroup = 2;       // units per A-buffer pair (the hand-over granularity)
-constexpr int kSmemLimit = 227 * 1024;
-constexpr int kSetHdr = 512;    // per chunk-group set: sigma_lo[64], column sums[64]
-constexpr int kURing = 4;       // U tiles (4 KiB each) in flight ahead of the epilogue
-constexpr int kMaxPairs = 3;    // A-buffer pairs in tensor memory (one batch row: 3)
-
-struct Ctl {
-  uint64_t sfull[kMaxStages], sempty[kMaxStages];
-  uint64_t ufull[kURing];
-  uint64_t aempty[kMaxPairs];   // A-buffer pair free again: the MMAs that read it completed
-  uint64_t accfull[2], zfull[2], drain[4];
-  uint64_t vfull;         // V rows of the first chunk group
-  uint32_t a_ready[kExpWarps];  // A-buffer pairs stored, per expander warp (a sum could let
-                                // a fast warp stand in for a slow one)
-  uint32_t acc_free[2];   // accumulator zeroed by the epilogue: +1 per epilogue warp per release
-  uint32_t tmem_base;
-  int abort;
-  int abort_snap;
-  int red_ok;
-  int amaxi[16 * kDecodeMaxBatch];   // max |Z| per column (float bits; values >= 0)
-  int zsum[16 * kDecodeMaxBatch];    // sum of q per column
-};
+constexpr int kSlots = 2;              // tensor-memory A slots per team
+constexpr int kNI = 3;                 // issuer warps (20 warps in all at batch <= 2: 96 registers each)
+constexpr int kBarZ = 4;               // named barriers: 4 = all warps but the copy warp, 5 = epilogue
+constexpr int kBarEpi = 5;
+constexpr float kQMax = 32512.0f;      // |q| <= 127 * 256: q = 256 hi + lo with hi, lo in int8
 
 template <int B>
 struct Cfg {
-  static constexpr int NB = 32 * B;                 // MMA N: [hi plane 16B | lo plane 16B]
-  static constexpr int ZB = NB * kTileCols;         // operand bytes of one chunk
-  // Tensor memory: two accumulators of NB columns (double buffered across segments),
-  // then the A-buffer ring, 64 columns (128 lanes x 256 bytes) per unit, in pairs.
-  static constexpr uint32_t ACOL0 = 2 * NB;
-  static constexpr int NPAIRS = (512 - 2 * NB) / (64 * kGroup);
+  static constexpr int NB = 32 * B;                 // MMA N: hi plane (16 B columns) | lo plane
+  static constexpr int NCOL = 16 * B;               // columns (b, j) of Z
   static constexpr int C = decode_chunks_per_segment(B);
-  static constexpr int COLS = C * kTileCols;        // columns of a chunk group
-  static constexpr int SET = kSetHdr + C * ZB;      // one chunk-group set
-  static constexpr int VSCR = COLS * kK * 2;        // V rows of a group (fp16)
-  static constexpr int XSCR = COLS * B * 2 + COLS * 4;   // x rows (fp16/bf16), then 1/s (fp32)
-  static constexpr int XSF = COLS * B * 4;          // x (.) 1/s of the group (fp32)
-  static constexpr int URING = kURing * kTileBytes; // U rows of a row tile (128 x 16 fp16) per slot
+  static constexpr int ZB = decode_chunk_operand_bytes(B);
+  static constexpr int SET = C * ZB;                // one activation set (operand planes only)
+  static constexpr int T = B <= 2 ? 3 : 2;          // teams of four warps
+  static constexpr int NACC = B == 1 ? 4 : 2;       // segment accumulators in tensor memory
+  static constexpr uint32_t ACOL0 = NACC * NB;      // first A-slot column (64 columns per slot)
+  static constexpr int WISS = 4 * T;                // issuer warps WISS .. WISS + kNI - 1
+  static constexpr int WEPI = 4 * T + kNI;          // epilogue warps WEPI .. WEPI + 3
+  static constexpr int WCTL = WEPI + 4;             // copy thread, tensor-memory owner (last warp)
+  static constexpr int THREADS = 32 * (WCTL + 1);
+  static constexpr int ZTHREADS = THREADS - 32;     // warps that build the first sets
   static constexpr int STAGE = C * kTileBytes;
-  static constexpr int CTL = static_cast<int>((sizeof(Ctl) + 127) / 128 * 128);
-  static constexpr int FIXED = 2 * SET + VSCR + XSCR + XSF + URING + CTL;
-  static constexpr int NS0 = (kSmemLimit - FIXED) / STAGE;
+  static constexpr int CTL = 8192;
+  // staging for the first group's x rows and 1/s (its V rows go to the second set slot)
+  static constexpr int STG = B * C * kTileCols * 2 + C * kTileCols * 4;
+  static constexpr int STG_AL = (STG + 1023) / 1024 * 1024;
+  static constexpr int FIXED = 2 * SET + CTL + STG_AL;
+  static constexpr int NS0 = (227 * 1024 - FIXED) / STAGE;
   static constexpr int NS = NS0 < kMaxStages ? NS0 : kMaxStages;
   static constexpr int SMEM = NS * STAGE + FIXED;
-  static_assert(NS >= 2, "sign ring too small");
-  static_assert(NPAIRS >= 2 && NPAIRS <= kMaxPairs, "A-buffer ring");
-  static_assert(XSCR % 128 == 0 && VSCR % 128 == 0 && XSF % 128 == 0, "scratch alignment");
+  static_assert(ACOL0 + T * kSlots * 64 <= 512, "tensor memory columns");
+  static_assert(NS >= 4, "sign ring too small");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  // each decode CTA allocates all 512 tensor-memory columns: two must never share an SM
+  static_assert(2 * (SMEM + 1024) > 228 * 1024, "two decode CTAs would fit one SM");
+  static_assert(THREADS <= 1024, "threads per CTA");
+  static_assert(ZTHREADS / 32 <= 20, "per-warp partials of the set builders");
+  static_assert(4 * (THREADS / kTileRows) * B * kTileRows * 4 + THREADS * 4 <= NS * STAGE,
+                "the reduction's scratch fits the drained sign stages");
+  static_assert(C * kTileCols * 32 <= SET, "the first group's V rows fit the second set slot");
 };
+
+struct Ctl {
+  uint64_t sfull[kMaxStages], sempty[kMaxStages];
+  uint64_t aempty[3][kSlots];   // a slot's MMAs completed (one commit per unit)
+  uint64_t accfull[4];          // a segment's MMAs completed (one commit per unit)
+  uint64_t zready[2];           // a set built by the epilogue warps (groups 1, 2, ...)
+  uint64_t drain[kNI];
+  uint64_t ready[3][kSlots];    // a slot's four quadrants stored (one arrival per team warp)
+  uint64_t acc_free[4];         // an accumulator read and zeroed (one arrival per epilogue warp)
+  uint64_t vstage, xstage;      // the first group's V rows and 1/s / its x rows, in shared memory
+  uint32_t tmem_base;
+  int abort;
+  int nred;                     // row tiles this CTA completed in the current counting round
+  int count_ok;                 // the epilogue finished without error: count the partials
+  int amax[2][64];              // per set slot and column: max |Z| (float bits, >= 0)
+  int csum[2][64];              // per set slot and column: the group's integer sum of q
+  float sig[2][64];             // per set slot and column: the quantisation step
+  float rlo[2][64];             // per set slot and column: 1 / step
+  int wpart[20][64];            // per warp and column: a set builder's partial max / sum
+};
+static_assert(sizeof(Ctl) <= 8192, "control block");
 
 struct Seg {
   int i, rt, kgA, len, cg;
+  int cgb;   // chunk group within block i
 };
 __device__ __forceinline__ Seg seg_of(int s, const DecodeParams& p, int C) {
   Seg g;
   g.cg = s / p.RT;
   g.rt = s - g.cg * p.RT;
   g.i = g.cg / p.NCB;
-  g.kgA = (g.cg - g.i * p.NCB) * C;
+  g.cgb = g.cg - g.i * p.NCB;
+  g.kgA = g.cgb * C;
   g.len = min(C, p.KG - g.kgA);
   return g;
 }
+// The segment after g (chunk-group-major numbering), without divisions.
+__device__ __forceinline__ void seg_next(Seg& g, const DecodeParams& p, int C) {
+  if (++g.rt == p.RT) {
+    g.rt = 0;
+    ++g.cg;
+    if (++g.cgb == p.NCB) {
+      g.cgb = 0;
+      ++g.i;
+    }
+    g.kgA = g.cgb * C;
+    g.len = min(C, p.KG - g.kgA);
+  }
+}
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+// The run of segments [s0, s1) of CTA `cta`.  With at most as many chunk groups as CTAs,
+// every group gets floor or ceil(grid / groups) CTAs and splits its RT segments evenly
+// among them, so no CTA spans two groups (building a group's activation set is paid
+// once per CTA); otherwise the segments are split contiguously and a CTA spans several
+// groups, whose sets after the first are built in the background.
+__device__ __forceinline__ void cta_range(const DecodeParams& p, int cta, int grid, int& s0, int& s1) {
+  const int NG = p.n * p.NCB;
+  if (NG <= grid) {
+    const int base = grid / NG, extra = grid - base * NG;
+    int g, w, k;
+    if (cta < extra * (base + 1)) {
+      g = cta / (base + 1);
+      w = cta - g * (base + 1);
+      k = base + 1;
+    } else {
+      const int c2 = cta - extra * (base + 1);
+      g = extra + c2 / base;
+      w = c2 - (g - extra) * base;
+      k = base;
+    }
+    s0 = g * p.RT + (w * p.RT) / k;
+    s1 = g * p.RT + ((w + 1) * p.RT) / k;
+  } else {
+    s0 = static_cast<int>(static_cast<long long>(cta) * p.segs / grid);
+    s1 = static_cast<int>(static_cast<long long>(cta + 1) * p.segs / grid);
+  }
 }
 
 __device__ __forceinline__ void store_y(void* y, int bf16, size_t idx, float v) {
   if (bf16) static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
   else static_cast<__half*>(y)[idx] = __float2half_rn(v);
 }
-__device__ __forceinline__ float x_at(const uint16_t* xr, int bf16, int idx) {
-  const uint16_t h = xr[idx];
+__device__ __forceinline__ float x_at(const void* x, int bf16, size_t idx) {
+  const uint16_t h = static_cast<const uint16_t*>(x)[idx];
   return bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
 }
-
 __device__ __forceinline__ void set_error(const DecodeParams& p, Ctl* ctl) {
   ctl->abort = 1;
   atomicOr(p.err, kErrTimeout);
 }
 
-// Byte addresses of a chunk group's inputs in the stack and in x.
-__device__ __forceinline__ const uint8_t* v_rows(const DecodeParams& p, const Seg& sg) {
-  return p.blocks + static_cast<size_t>(sg.i) * p.block_bytes + static_cast<size_t>(p.m) * p.d / 8 +
-         static_cast<size_t>(2) * kK * p.m + static_cast<size_t>(sg.kgA) * kTileCols * kK * 2;
+// Byte offsets inside one block record.
+__device__ __forceinline__ const uint8_t* record(const DecodeParams& p, int i) {
+  return p.blocks + static_cast<size_t>(i) * p.block_bytes;
 }
-__device__ __forceinline__ const uint8_t* u_tile(const DecodeParams& p, int i, int rt) {
-  return p.blocks + static_cast<size_t>(i) * p.block_bytes + static_cast<size_t>(p.m) * p.d / 8 +
-         static_cast<size_t>(rt) * kTileRows * kK * 2;
-}
-
-// Loads the inputs of chunk group `sg` into the scratch with plain loads (the later
-// groups of a CTA; the first one arrives by bulk copies).  Called by the 128 epilogue
-// threads after griddep_wait.
-template <int B>
-__device__ void load_set_inputs(const DecodeParams& p, uint8_t* vscr, uint8_t* xscr, const Seg& sg, int tid) {
-  using K = Cfg<B>;
-  const int cols = sg.len * kTileCols, col0 = sg.kgA * kTileCols;
-  const uint4* vsrc = reinterpret_cast<const uint4*>(v_rows(p, sg));
-  for (int v = tid; v < cols * 2; v += 128) reinterpret_cast<uint4*>(vscr)[v] = __ldg(vsrc + v);
-  uint16_t* xr = reinterpret_cast<uint16_t*>(xscr);
-  for (int idx = tid; idx < B * cols; idx += 128) {
-    const int b = idx / cols, c = idx - b * cols;
-    xr[b * K::COLS + c] = static_cast<const uint16_t*>(p.x)[static_cast<size_t>(b) * p.d + col0 + c];
-  }
-  float* isv = reinterpret_cast<float*>(xscr + K::COLS * B * 2);
-  for (int c = tid; c < cols; c += 128) isv[c] = __ldg(p.inv_s + col0 + c);
+__device__ __forceinline__ size_t u_offset(const DecodeParams& p) { return static_cast<size_t>(p.m) * p.d / 8; }
+__device__ __forceinline__ size_t v_offset(const DecodeParams& p) {
+  return u_offset(p) + static_cast<size_t>(2) * kK * p.m;
 }
 
-// Quantises the activation chunks of chunk group `sg` (inputs already in the scratch:
-// V rows, x rows, 1/s) into `set`: operand planes in the UMMA no-swizzle K-major
-// layout, the per-column step sigma_lo and the dequantised column sum.  Run by NT
-// threads that share named barrier `bar`; it has no other wait, so every thread passes
-// the same barriers.  `zfull` is signalled unless `skip`.
-template <int B, int NT>
-__device__ void produce_set(uint8_t* set, const uint8_t* vscr, const uint8_t* xscr, float* xsf, int bf16, Ctl* ctl,
-                            const Seg& sg, int tid, int bar, uint64_t* zfull, bool skip) {
-  using K = Cfg<B>;
-  const int cols = sg.len * kTileCols;
-  const __half* vh = reinterpret_cast<const __half*>(vscr);
-  const uint16_t* xr = reinterpret_cast<const uint16_t*>(xscr);
-  const float* isv = reinterpret_cast<const float*>(xscr + K::COLS * B * 2);
-  // x' = x (.) 1/s, once per column and batch row
-  for (int idx = tid; idx < B * cols; idx += NT) {
-    const int b = idx / cols, c = idx - b * cols;
-    xsf[b * K::COLS + c] = __fmul_rn(x_at(xr, bf16, b * K::COLS + c), isv[c]);
-  }
-  named_sync(bar, NT);
-  const int items = (cols / 16) * 16 * B;   // (16-column group, column (b, j)), column fastest
-  if (!skip) {
-    // pass 1: max |Z| per column over the group; a thread folds its items of one
-    // column before touching shared memory
-    int lcol = -1;
-    float lmx = 0.0f;
-    for (int it = tid; it < items; it += NT) {
-      const int c16 = it / (16 * B), col = it - c16 * 16 * B;
-      const int b = col >> 4, j = col & 15;
-      const float* xp = xsf + b * K::COLS + c16 * 16;
-      const __half* vp = vh + c16 * 16 * kK + j;
-      float mx = 0.0f;
+// K-step t of a unit from one sign word: bit t of every byte moved to bit 7 and the
+// rest cleared, i.e. the s8 operand -128 * Sb.  The shift is a multiply, which runs on
+// the FMA pipe; only the AND takes the (half-rate) integer pipe.
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t w, int t) {
+  uint32_t v = w;
+  if (t < 7) asm("mul.lo.u32 %0, %1, %2;" : "=r"(v) : "r"(w), "r"(1u << (7 - t)));
+  return v & 0x80808080u;
+}
+
+// The quantisation step of a column from the largest |Z| of its chunk group.
+__device__ __forceinline__ float step_of(float amax) {
+  return amax > 0.0f ? __fmul_rn(amax, 1.0f / kQMax) : 1.0f;
+}
+
+// Reduce-scatter of 16 values over the 32 lanes of a warp (pairwise exchanges, 16
+// shuffles): afterwards lane l holds, in its return value, the reduction over all
+// lanes of value index scatter_index(l); lanes l and l ^ 1 hold the same index.
+__device__ __forceinline__ int scatter_index(int lane) {
+  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
+template <typename Tv, typename Op>
+__device__ __forceinline__ Tv warp_reduce_scatter16(Tv (&v)[16], int lane, Op op) {
+  constexpr uint32_t FULL = 0xffffffffu;
 #pragma unroll
-      for (int kin = 0; kin < 16; ++kin) mx = fmaxf(mx, fabsf(__fmul_rn(xp[kin], __half2float(vp[kin * kK]))));
-      if (col != lcol) {
-        if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
-        lcol = col;
-        lmx = mx;
-      } else {
-        lmx = fmaxf(lmx, mx);
-      }
-    }
-    if (lcol >= 0) atomicMax(&ctl->amaxi[lcol], __float_as_int(lmx));
+  for (int e = 0; e < 8; ++e) {
+    const bool up = (lane & 16) != 0;
+    const Tv send = up ? v[e] : v[e + 8], keep = up ? v[e + 8] : v[e];
+    v[e] = op(keep, __shfl_xor_sync(FULL, send, 16));
   }
-  named_sync(bar, NT);
-  if (!skip) {
-    // pass 2: q = rint(Z / sigma_lo), |q| <= 127 * 256, q = 256 hi + lo
-    uint8_t* ops = set + kSetHdr;
-    int lcol = -1, lsum = 0;
-    float rlo = 1.0f;
-    for (int it = tid; it < items; it += NT) {
-      const int c16 = it / (16 * B), col = it - c16 * 16 * B;
-      const int b = col >> 4, j = col & 15;
-      if (col != lcol) {
-        if (lcol >= 0) atomicAdd(&ctl->zsum[lcol], lsum);
-        lcol = col;
-        lsum = 0;
-        const float amax = __int_as_float(ctl->amaxi[col]);
-        const float slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
-        rlo = 1.0f / slo;
-      }
-      const float* xp = xsf + b * K::COLS + c16 * 16;
-      const __half* vp = vh + c16 * 16 * kK + j;
-      uint32_t hw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int kin = 0; kin < 16; ++kin) {
-        const float z = __fmul_rn(xp[kin], __half2float(vp[kin * kK]));
-        int qv = __float2int_rn(z * rlo);
-        qv = max(-32512, min(32512, qv));
-        const int qh = (qv + 128) >> 8;
-        const int ql = qv - (qh << 8);
-        lsum += qv;
-        hw[kin >> 2] |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * (kin & 3));
-        lw[kin >> 2] |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * (kin & 3));
+  for (int e = 0; e < 4; ++e) {
+    const bool up = (lane & 8) != 0;
+    const Tv send = up ? v[e] : v[e + 4], keep = up ? v[e + 4] : v[e];
+    v[e] = op(keep, __shfl_xor_sync(FULL, send, 8));
+  }
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const bool up = (lane & 4) != 0;
+    const Tv send = up ? v[e] : v[e + 2], keep = up ? v[e + 2] : v[e];
+    v[e] = op(keep, __shfl_xor_sync(FULL, send, 4));
+  }
+  {
+    const bool up = (lane & 2) != 0;
+    const Tv send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+    v[0] = op(keep, __shfl_xor_sync(FULL, send, 2));
+  }
+  return op(v[0], __shfl_xor_sync(FULL, v[0], 1));
+}
+struct MaxOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct AddOp {
+  __device__ __forceinline__ int operator()(int a, int b) const { return a + b; }
+};
+
+// The 16 fp16 entries of one V row (32 bytes) as fp32, from global memory (read-only
+// path) or from shared memory.
+template <bool kGlobal>
+__device__ __forceinline__ void v_row(const uint8_t* row, float (&v)[16]) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  const uint4 a = kGlobal ? __ldg(r4) : r4[0], b = kGlobal ? __ldg(r4 + 1) : r4[1];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+    v[2 * e] = f.x;
+    v[2 * e + 1] = f.y;
+  }
+}
+
+// Input columns of chunk group cg: block i, columns [col0, col0 + gcols).
+struct Group {
+  int i, col0, gcols;
+};
+__device__ __forceinline__ Group group_of(const DecodeParams& p, int cg, int C) {
+  Group g;
+  g.i = cg / p.NCB;
+  const int k0 = (cg - g.i * p.NCB) * C;
+  g.col0 = k0 * kTileCols;
+  g.gcols = min(C, p.KG - k0) * kTileCols;
+  return g;
+}
+
+// Where a set builder reads the group's inputs: V row of group column c at v + 32 c,
+// x[b] at x[b * xs + c], 1/s at is[c] -- global memory for sets built in the
+// background, shared-memory copies (bulk-copied by the copy thread) for the first set.
+struct SetSrc {
+  const uint8_t* v;
+  const uint16_t* x;
+  const float* is;
+  int xs;
+};
+
+// The activation set of chunk group cg is built in two passes by NT threads (index
+// zt, whole warps) that share a named barrier; thread zt owns group columns zt,
+// zt + NT, ... (whole V rows):
+//   set_max    Z = (x (.) 1/s) (.) V_i over its columns, max |Z| per column (b, j);
+//   set_quant  q = rint(Z / sigma), sigma = max |Z| / 32512, into the operand layout
+//              as the two int8 planes q = 256 hi + lo, and the integer sums of q;
+// with ctl->{amax, csum, sig}[slot] as the shared state.  Per-column maxima and sums
+// are warp reduce-scatters and one shared atomic per column and warp.
+template <bool kGlobal>
+__device__ __forceinline__ float x_scaled(const DecodeParams& p, const SetSrc& S, int c, int b) {
+  const uint16_t h = S.x[b * S.xs + c];
+  const float xv = p.x_bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
+  return __fmul_rn(xv, kGlobal ? __ldg(S.is + c) : S.is[c]);
+}
+
+template <int B, bool kGlobal>
+__device__ void set_max(const DecodeParams& p, Ctl* ctl, int slot, const SetSrc& S, int gcols, int zt, int NT) {
+  const int lane = zt & 31;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float mx[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) mx[jj] = 0.0f;
+    for (int c = zt; c < gcols; c += NT) {
+      const float xv = x_scaled<kGlobal>(p, S, c, b);
+      float v[16];
+      v_row<kGlobal>(S.v + static_cast<size_t>(c) * 32, v);
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) mx[jj] = fmaxf(mx[jj], fabsf(__fmul_rn(xv, v[jj])));
+    }
+    const float m = warp_reduce_scatter16(mx, lane, MaxOp());
+    if ((lane & 1) == 0) ctl->wpart[zt >> 5][b * 16 + scatter_index(lane)] = __float_as_int(m);
+  }
+}
+
+template <int B, bool kGlobal>
+__device__ void set_quant(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
+                          int NT) {
+  using K = Cfg<B>;
+  constexpr int NB = K::NB, NCOL = K::NCOL;
+  const int lane = zt & 31;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    const float* rlo = ctl->rlo[slot] + b * 16;   // shared-memory broadcast reads
+    int zs[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) zs[jj] = 0;
+    for (int c = zt; c < gcols; c += NT) {
+      const float xv = x_scaled<kGlobal>(p, S, c, b);
+      float v[16];
+      v_row<kGlobal>(S.v + static_cast<size_t>(c) * 32, v);
+      // operand layout: no-swizzle K-major core matrices of 8 operand columns x 16 K;
+      // K-step t at t * NB * 32, core matrices adjacent in K 128 bytes apart, in N 256
+      const int cc = c >> 8, cl = c & 255;
+      uint8_t* base = set + cc * K::ZB + ((cl >> 5) * (NB / 8) * 2 + ((cl >> 4) & 1)) * 128 + (cl & 15);
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        // |Z| / sigma <= 32512 up to a rounding far below 1/2, so rint stays in range
+        const int q = __float2int_rn(__fmul_rn(xv, v[jj]) * rlo[jj]);
+        zs[jj] += q;
+        const int nh = b * 16 + jj, nl = NCOL + nh;
+        base[(nh >> 3) * 256 + (nh & 7) * 16] = static_cast<uint8_t>((q + 128) >> 8);   // hi
+        base[(nl >> 3) * 256 + (nl & 7) * 16] = static_cast<uint8_t>(q);                // lo = q - 256 hi, mod 256
       }
-      // chunk cc, K-step t (32 columns), K half kc, 8-row core matrix n / 8
-      const int cc = c16 >> 4, g16 = c16 & 15;
-      const int t = g16 >> 1, kc = g16 & 1;
-      const int nh = col, nl = 16 * B + col;
-      uint8_t* base = ops + static_cast<size_t>(cc) * K::ZB;
-      *reinterpret_cast<uint4*>(base + ((t * (K::NB / 8) + nh / 8) * 2 + kc) * 128 + (nh % 8) * 16) =
-          make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(base + ((t * (K::NB / 8) + nl / 8) * 2 + kc) * 128 + (nl % 8) * 16) =
-          make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    if (lcol >= 0) atomicAdd(&ctl->zsum[lcol], lsum);
-    fence_proxy_async_smem();   // the MMAs read the operands through the async proxy
+    const int sum = warp_reduce_scatter16(zs, lane, AddOp());
+    if ((lane & 1) == 0) ctl->wpart[zt >> 5][b * 16 + scatter_index(lane)] = sum;
   }
-  named_sync(bar, NT);
-  if (tid < 16 * B) {
-    if (!skip) {
-      const float amax = __int_as_float(ctl->amaxi[tid]);
-      const float slo = amax > 0.0f ? __fmul_rn(amax, 1.0f / 32512.0f) : 1.0f;
-      float* hdr = reinterpret_cast<float*>(set);
-      hdr[tid] = slo;
-      hdr[64 + tid] = __fmul_rn(slo, static_cast<float>(ctl->zsum[tid]));
-    }
-    ctl->amaxi[tid] = 0;
-    ctl->zsum[tid] = 0;
+}
+
+template <int B, bool kGlobal>
+__device__ void build_set(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
+                          int NT, int bar) {
+  constexpr int NCOL = Cfg<B>::NCOL;
+  const int nw = NT >> 5;
+  // pass 1; each warp leaves its per-column maxima in wpart, then one thread per column
+  // folds them (no two warps update one shared word)
+  set_max<B, kGlobal>(p, ctl, slot, S, gcols, zt, NT);
+  bar_named(bar, NT);
+  if (zt < NCOL) {
+    int m = 0;
+    for (int w = 0; w < nw; ++w) m = max(m, ctl->wpart[w][zt]);   // max |Z| as float bits, all >= 0
+    ctl->amax[slot][zt] = m;
+    const float sg = step_of(__int_as_float(m));
+    ctl->sig[slot][zt] = sg;
+    ctl->rlo[slot][zt] = 1.0f / sg;
   }
-  named_sync(bar, NT);
-  if (tid == 0 && !skip) mbar_arrive(zfull);
+  bar_named(bar, NT);
+  set_quant<B, kGlobal>(p, ctl, slot, set, S, gcols, zt, NT);
+  fence_proxy_async_smem();   // the MMAs read the operand through the async proxy
+  bar_named(bar, NT);
+  if (zt < NCOL) {
+    int sum = 0;
+    for (int w = 0; w < nw; ++w) sum += ctl->wpart[w][zt];
+    ctl->csum[slot][zt] = sum;
+  }
+  bar_named(bar, NT);
+}
+
+// A set built from global memory (the epilogue warps, in the background).
+template <int B>
+__device__ void build_set_global(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, int cg, int zt, int NT,
+                                 int bar) {
+  const Group G = group_of(p, cg, Cfg<B>::C);
+  SetSrc S;
+  S.v = record(p, G.i) + v_offset(p) + static_cast<size_t>(G.col0) * 32;
+  S.x = static_cast<const uint16_t*>(p.x) + G.col0;
+  S.is = p.inv_s + G.col0;
+  S.xs = p.d;
+  build_set<B, true>(p, ctl, slot, set, S, G.gcols, zt, NT, bar);
+}
+
+// MMA issued by the elected lane of a warp whose lanes hold the same operands.
+__device__ __forceinline__ void mma_i8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+__device__ __forceinline__ void commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 template <int B>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const DecodeParams p) {
   using K = Cfg<B>;
-  constexpr int NB = K::NB, C = K::C, NS = K::NS, NPAIRS = K::NPAIRS;
-  constexpr uint32_t IDESC = make_idesc(2u, 0u, 1u, 128u, NB);  // s32 <- u8 x s8, M=128, N=NB
+  constexpr int NB = K::NB, NCOL = K::NCOL, C = K::C, NS = K::NS, T = K::T, NACC = K::NACC;
+  constexpr uint32_t IDESC = make_idesc(2u, 1u, 1u, 128u, NB);   // s32 <- s8 x s8, M = 128, N = NB
+  constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* stages = smem;
-  uint8_t* sets = smem + NS * K::STAGE;
-  uint8_t* vscr = sets + 2 * K::SET;
-  uint8_t* xscr = vscr + K::VSCR;
-  float* xsf = reinterpret_cast<float*>(xscr + K::XSCR);
-  uint8_t* uring = xscr + K::XSCR + K::XSF;
-  Ctl* ctl = reinterpret_cast<Ctl*>(uring + K::URING);
+  uint8_t* sets = smem;                              // 2 activation sets (1024-aligned)
+  uint8_t* stages = smem + 2 * K::SET;               // sign stages
+  Ctl* ctl = reinterpret_cast<Ctl*>(stages + NS * K::STAGE);
+  uint8_t* stg = reinterpret_cast<uint8_t*>(ctl) + K::CTL;   // first group: x rows, then 1/s
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x, grid = gridDim.x;
-  const int s0 = static_cast<int>(static_cast<long long>(cta) * p.segs / grid);
-  const int s1 = static_cast<int>(static_cast<long long>(cta + 1) * p.segs / grid);
+  int s0, s1;
+  cta_range(p, cta, grid, s0, s1);
   const int nseg = s1 - s0;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
-  const int NC = p.n * p.NCB;   // chunk groups = partials per row tile
   const Seg sg0 = seg_of(s0, p, C);
+  const int last_cg = seg_of(s1 - 1, p, C).cg;
+  const int NZ = last_cg - sg0.cg + 1;               // chunk groups this CTA touches (consecutive)
 
   griddep_launch_dependents();
 
   // ------------------------------------------------------------------ set-up -----
-  if (warp == kWarpCopy) {
+  if (warp == K::WCTL) {
     tmem_alloc(&ctl->tmem_base, 512);
     if (lane == 0) {
-      for (int s = 0; s < kMaxStages; ++s) {
+      for (int s = 0; s < NS; ++s) {
         mbar_init(&ctl->sfull[s], 1);
-        mbar_init(&ctl->sempty[s], kExpWarps);
+        mbar_init(&ctl->sempty[s], 4 * C);          // four warps per unit, C units per stage
       }
-      for (int u = 0; u < kURing; ++u) mbar_init(&ctl->ufull[u], 1);
-      for (int q = 0; q < kMaxPairs; ++q) mbar_init(&ctl->aempty[q], kNI);
-      for (int q = 0; q < 2; ++q) {
-        mbar_init(&ctl->accfull[q], kNI);
-        mbar_init(&ctl->zfull[q], 1);
+      for (int t = 0; t < 3; ++t)
+        for (int q = 0; q < kSlots; ++q) {
+          mbar_init(&ctl->aempty[t][q], 1);
+          mbar_init(&ctl->ready[t][q], 4);
+        }
+      for (int a = 0; a < 4; ++a) {
+        mbar_init(&ctl->accfull[a], C);              // one commit per unit
+        mbar_init(&ctl->acc_free[a], 4);
       }
-      for (int w = 0; w < 4; ++w) mbar_init(&ctl->drain[w], 1);
-      mbar_init(&ctl->vfull, 1);
+      mbar_init(&ctl->vstage, 1);
+      mbar_init(&ctl->xstage, 1);
+      for (int z = 0; z < 2; ++z) mbar_init(&ctl->zready[z], 1);
+      for (int w = 0; w < kNI; ++w) mbar_init(&ctl->drain[w], 1);
       ctl->abort = 0;
-      for (int w = 0; w < kExpWarps; ++w) ctl->a_ready[w] = 0;
-      ctl->acc_free[0] = 0;
-      ctl->acc_free[1] = 0;
-      for (int c = 0; c < 16 * kDecodeMaxBatch; ++c) {
-        ctl->amaxi[c] = 0;
-        ctl->zsum[c] = 0;
-      }
+      ctl->nred = 0;
+      ctl->count_ok = 0;
       fence_barrier_init();
     }
   }
@@ -330,377 +480,369 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp < kExpWarps) {
-    // ------------------------------------------------ expanders (rows = lanes) -----
-    // Units are walked in order in pairs: pair g goes to A-buffer pair g mod NPAIRS and
-    // is expanded by team g & 1 (warps 0-3 or 4-7; warp % 4 is the TMEM lane quadrant).
-    // Every expander warp walks all units (so all agree on the sign stages, each of
-    // which all eight release) but expands only its team's pairs; warp e adds 1 to
-    // a_ready[e] (release) once its rows of a pair are in tensor memory, and the
-    // issuers wait for the four warps of the pair's team.  A warp whose wait ran out
-    // stops signalling (the issuers' bounded waits then run out too); failure is
-    // decided per warp by vote.
-    const int team = warp >> 2;
-    const int tid = (warp & 3) * 32 + lane;   // row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    bool failed = false;
-    auto check = [&](bool ok) {
-      if (!__all_sync(0xffffffffu, ok)) failed = true;
-    };
-    int j = 0, c = 0, waited = -1;
-    Seg sg = sg0;
-    for (int g = 0; j < nseg && !failed; ++g) {
-      const int pr = g % NPAIRS;
-      const bool mine = (g & 1) == team;
-      if (mine && g >= NPAIRS)
-        check(mbar_wait(&ctl->aempty[pr], static_cast<uint32_t>((g / NPAIRS - 1) & 1), deadline, abort_flag));
-      for (int q = 0; q < kGroup && j < nseg && !failed; ++q) {
-        const int st = j % NS;
-        if (mine) {
-          if (waited != j) {
-            check(mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag));
-            waited = j;
+  if (warp == K::WCTL) {
+    // ------------------------------------------------------------- copy thread -------
+    if (lane == 0) {
+      Seg sc = sg0;   // the segment of the next stage to issue (stages are issued in order)
+      auto issue_stage = [&](int jj) {
+        const Seg sg = sc;
+        seg_next(sc, p, C);
+        const int st = jj % NS;
+        const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
+        mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
+        bulk_g2s(stages + st * K::STAGE,
+                 record(p, sg.i) + (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes, bytes, &ctl->sfull[st]);
+      };
+      // The first group's V rows (into the second set slot) and 1/s, then the sign tiles:
+      // stack memory and the scale vector, read before the previous kernel has finished.
+      // (Timeout test: CTA 0 leaves out its first stage, so its waits run out while the
+      // other CTAs complete and count their partials.)
+      const Group G0 = group_of(p, sg0.cg, C);
+      mbar_arrive_expect_tx(&ctl->vstage, static_cast<uint32_t>(G0.gcols) * 36u);
+      bulk_g2s(sets + K::SET, record(p, G0.i) + v_offset(p) + static_cast<size_t>(G0.col0) * 32,
+               static_cast<uint32_t>(G0.gcols) * 32u, &ctl->vstage);
+      bulk_g2s(stg + B * C * kTileCols * 2, p.inv_s + G0.col0, static_cast<uint32_t>(G0.gcols) * 4u, &ctl->vstage);
+      const bool skip_first = p.inject_unreachable && cta == 0;
+      int issued = 0;
+      for (; issued < NS && issued < nseg; ++issued) {
+        if (skip_first && issued == 0) {
+          seg_next(sc, p, C);
+          continue;
+        }
+        issue_stage(issued);
+      }
+      // x only after the kernel ahead has finished (it may have written x)
+      griddep_wait();
+      mbar_arrive_expect_tx(&ctl->xstage, static_cast<uint32_t>(B * G0.gcols) * 2u);
+      for (int b = 0; b < B; ++b)
+        bulk_g2s(stg + b * C * kTileCols * 2, static_cast<const uint16_t*>(p.x) + static_cast<size_t>(b) * p.d + G0.col0,
+                 static_cast<uint32_t>(G0.gcols) * 2u, &ctl->xstage);
+      bool ok = true;
+      for (; ok && issued < nseg; ++issued) {
+        ok = mbar_wait(&ctl->sempty[issued % NS], static_cast<uint32_t>((issued / NS - 1) & 1), deadline, abort_flag);
+        if (ok) issue_stage(issued);
+        else break;
+      }
+      if (!ok) set_error(p, ctl);
+      // no copy may still be landing in shared memory when the CTA exits
+      const uint64_t drain_by = globaltimer_ns() + 100000000ull;
+      for (int e = (issued > NS ? issued - NS : 0); e < issued; ++e) {
+        if (skip_first && e == 0) continue;
+        mbar_wait(&ctl->sfull[e % NS], static_cast<uint32_t>((e / NS) & 1), drain_by, nullptr);
+      }
+      mbar_wait(&ctl->vstage, 0, drain_by, nullptr);
+      mbar_wait(&ctl->xstage, 0, drain_by, nullptr);
+    }
+  } else {
+    // ---- every other warp: build the first activation set together --------------------
+    {
+      const int zt = threadIdx.x;   // 0 .. ZTHREADS - 1
+      // warm L2 with the V rows of the second group (stack memory, read before the kernel
+      // ahead has finished); the first group's inputs arrive in shared memory
+      if (NZ > 1) {
+        const Group G = group_of(p, sg0.cg + 1, C);
+        for (int c = zt; c < G.gcols; c += K::ZTHREADS)
+          prefetch_l2(record(p, G.i) + v_offset(p) + static_cast<size_t>(G.col0 + c) * 32);
+      }
+      griddep_wait();   // the workspace, y and x belong to this launch only from here on
+      bool ok = mbar_wait(&ctl->vstage, 0, deadline, abort_flag);
+      ok = ok && mbar_wait(&ctl->xstage, 0, deadline, abort_flag);
+      if (!ok) set_error(p, ctl);   // the set is then garbage; every later wait sees the abort flag
+      const Group G0 = group_of(p, sg0.cg, C);
+      SetSrc S;
+      S.v = sets + K::SET;
+      S.x = reinterpret_cast<const uint16_t*>(stg);
+      S.is = reinterpret_cast<const float*>(stg + B * C * kTileCols * 2);
+      S.xs = C * kTileCols;
+      build_set<B, false>(p, ctl, 0, sets, S, G0.gcols, zt, K::ZTHREADS, kBarZ);
+    }
+
+    if (warp < K::WISS) {
+      // ---------------------------------- teams: expand signs into tensor memory -----
+      const int team = warp >> 2, q = warp & 3;
+      const int tid = 32 * q + lane;                              // row of the unit = TMEM lane
+      const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+      int j = 0, c = 0, u = 0, k = 0;
+      Seg sg = sg0;
+      while (j < nseg) {
+        if (u % T == team) {
+          const int slot = k % kSlots, use = k / kSlots;
+          const int st = j % NS;
+          bool ok = true;
+          if (use > 0) ok = mbar_wait(&ctl->aempty[team][slot], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
+          if (ok) ok = mbar_wait(&ctl->sfull[st], static_cast<uint32_t>((j / NS) & 1), deadline, abort_flag);
+          ok = __all_sync(FULL, ok);
+          if (!ok) {
+            set_error(p, ctl);
+            break;
           }
-          if (failed) break;
           const uint8_t* tile = stages + st * K::STAGE + c * kTileBytes;
           const uint4 wa = *reinterpret_cast<const uint4*>(tile + tid * 16);
           const uint4 wb = *reinterpret_cast<const uint4*>(tile + 2048 + tid * 16);
           const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-          const uint32_t abase = tmem + lane_base + K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
-          // K-step t holds bit t of every byte of the unit's words: byte q of word pw is
-          // sign column 32 t + 4 pw + q (the device tile order), value 0 or 1
+          const uint32_t acol = K::ACOL0 + 64u * static_cast<uint32_t>(team * kSlots + slot);
+          // byte q of word pw is sign column 32 t + 4 pw + q in bit t: K-step t of the
+          // unit is bit t of every byte (the device tile order), moved to bit 7
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t r[32];
 #pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
+            for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
-              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = (w[pw] >> (4 * h + tt)) & 0x01010101u;
-            }
-            tmem_st32(abase + 32 * h, r);
+              for (int pw = 0; pw < 8; ++pw) r[tt * 8 + pw] = sign_bytes(w[pw], 4 * h + tt);
+            tmem_st32(tmem + lane_base + acol + 32u * h, r);
           }
-        }
-        if (++c == sg.len) {
-          // segment done (its words are in registers): release the stage to the copy warp
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl->sempty[st]);
+          if (lane == 0) {   // this warp's rows of the stage are in registers
+            mbar_arrive(&ctl->sempty[st]);
+            if (c == sg.len - 1)
+              for (int e = sg.len; e < C; ++e) mbar_arrive(&ctl->sempty[st]);
+          }
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->ready[team][slot]);
+          ++k;
+        }
+        ++u;
+        if (++c == sg.len) {
           c = 0;
           ++j;
-          if (j < nseg) sg = seg_of(s0 + j, p, C);
+          seg_next(sg, p, C);
         }
       }
-      if (failed) break;
-      if (mine) {
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) red_release_shared_add(&ctl->a_ready[warp], 1u);
+    } else if (warp < K::WEPI) {
+      // ------------------------------------------ MMA issuers (warp-uniform, elect) -----
+      const int w = warp - K::WISS;
+      int j = 0, c = 0, u = 0, zk = 0, waited_zk = 0, checked_j = -1;
+      bool ok = true, any = false;
+      Seg sg = sg0;
+      while (j < nseg && ok) {
+        if (u % kNI == w) {
+          const int team = u % T, k = u / T, slot = k % kSlots, use = k / kSlots;
+          const int a = j % NACC;
+          // the slot's four quadrants are stored
+          ok = mbar_wait(&ctl->ready[team][slot], static_cast<uint32_t>(use & 1), deadline, abort_flag);
+          // the sets of groups 1, 2, ... are built by the epilogue warps
+          if (ok && zk > waited_zk) {
+            ok = mbar_wait(&ctl->zready[zk & 1], static_cast<uint32_t>(((zk - 1) >> 1) & 1), deadline, abort_flag);
+            waited_zk = zk;
+          }
+          // the segment's accumulator has been read and zeroed
+          if (ok && checked_j != j) {
+            ok = mbar_wait(&ctl->acc_free[a], static_cast<uint32_t>((j / NACC) & 1), deadline, abort_flag);
+            checked_j = j;
+          }
+          ok = __all_sync(FULL, ok);
+          if (!ok) break;
+          tc_fence_after();
+          // K-step t of the chunk starts t * NB * 32 bytes further (the descriptor's address
+          // field counts 16-byte units; shared-memory addresses stay below 256 KB)
+          const uint64_t bdesc0 = smem_desc_noswizzle(smem_u32(sets + (zk & 1) * K::SET + c * K::ZB), 128, 256);
+          const uint32_t adst = tmem + static_cast<uint32_t>(a * NB);
+          const uint32_t asrc = tmem + K::ACOL0 + 64u * static_cast<uint32_t>(team * kSlots + slot);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            mma_i8_elect(adst, asrc + 8u * t, bdesc0 + static_cast<uint64_t>((t * (NB / 8) * 256) >> 4), IDESC);
+          commit_elect(&ctl->aempty[team][slot]);
+          commit_elect(&ctl->accfull[a]);
+          if (c == sg.len - 1 && lane == 0)
+            for (int e = sg.len; e < C; ++e) mbar_arrive(&ctl->accfull[a]);
+          any = true;
+        }
+        ++u;
+        if (++c == sg.len) {
+          c = 0;
+          ++j;
+          const int cg = sg.cg;
+          seg_next(sg, p, C);
+          if (sg.cg != cg) ++zk;
+        }
       }
-    }
-    if (failed) set_error(p, ctl);
-  } else if (warp < kWarpIss0 + 4) {
-    // --------- warps 8-15: the first chunk group's activation chunks, together ------
-    const int tp = threadIdx.x - kWarpEpi0 * 32;   // 0..255
-    bool pfailed = false;
-    if (warp < kWarpIss0) {
-      // accumulators start at zero (the MMAs only accumulate); release both
-      const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
+      if (!ok) set_error(p, ctl);
+      if (any) {   // no MMA may still read or write tensor memory at exit
+        commit_elect(&ctl->drain[w]);
+        mbar_wait(&ctl->drain[w], 0, globaltimer_ns() + 100000000ull, nullptr);
+      }
+    } else {
+      // ------------------------------------- epilogue, partials, row-tile reduction -----
+      const int q = warp & 3;
+      const int et = threadIdx.x - 32 * K::WEPI;                   // 0 .. 127
+      const int tid = 32 * q + lane;                               // row of the tile = TMEM lane
+      const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+      const int NC = p.n * p.NCB;                                  // partials per row tile
       uint32_t zr[32];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) zr[q] = 0u;
+      for (int e = 0; e < 32; ++e) zr[e] = 0u;
+      // accumulators start at zero (the MMAs only accumulate): zero and release them all
 #pragma unroll
-      for (int cc = 0; cc < 2 * NB; cc += 32) tmem_st32(tmem + lane_base + cc, zr);
+      for (int cc = 0; cc < NACC * NB; cc += 32) tmem_st32(tmem + lane_base + cc, zr);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        red_release_shared_add(&ctl->acc_free[0], 1u);
-        red_release_shared_add(&ctl->acc_free[1], 1u);
+      if (lane == 0)
+        for (int a = 0; a < NACC; ++a) mbar_arrive(&ctl->acc_free[a]);
+      // the CTA's second chunk group (if any) is built here, while the teams and issuers
+      // work through the first
+      if (NZ > 1) {
+        build_set_global<B>(p, ctl, 1, sets + K::SET, sg0.cg + 1, et, 128, kBarEpi);
+        if (et == 0) mbar_arrive(&ctl->zready[1]);
       }
-    }
-    if (nseg > 0) {
-      // x and 1/s of the first group by plain loads (only after the previous kernel in
-      // the stream has finished: it may have written them), V rows by a bulk copy
-      griddep_wait();
-      {
-        const int cols = sg0.len * kTileCols, col0 = sg0.kgA * kTileCols;
-        uint16_t* xr = reinterpret_cast<uint16_t*>(xscr);
-        for (int idx = tp; idx < B * cols; idx += 256) {
-          const int b = idx / cols, c = idx - b * cols;
-          xr[b * K::COLS + c] = static_cast<const uint16_t*>(p.x)[static_cast<size_t>(b) * p.d + col0 + c];
-        }
-        float* isv = reinterpret_cast<float*>(xscr + K::COLS * B * 2);
-        for (int c = tp; c < cols; c += 256) isv[c] = __ldg(p.inv_s + col0 + c);
-      }
-      const bool ok = mbar_wait(&ctl->vfull, 0, deadline, abort_flag);
-      pfailed = !__all_sync(0xffffffffu, ok);
-      // a warp that timed out still runs the set's barriers, skipping the work; the
-      // others see the abort flag it set
-      if (pfailed) set_error(p, ctl);
-      named_sync(kBarProd, 256);
-      produce_set<B, 256>(sets, vscr, xscr, xsf, p.x_bf16, ctl, sg0, tp, kBarProd, &ctl->zfull[0],
-                          *abort_flag != 0);
-    }
-    if (warp < kWarpIss0) {
-      // ------------------------------- epilogue, later chunk groups, row tiles -----
-      const int tid = threadIdx.x - kWarpEpi0 * 32;   // row within the tile = TMEM lane
-      const uint32_t lane_base = static_cast<uint32_t>((warp - kWarpEpi0) * 32) << 16;
-      bool failed = pfailed;
-      auto check = [&](bool ok) {
-        if (!__all_sync(0xffffffffu, ok)) failed = true;
-      };
-      griddep_wait();   // the workspace and y belong to this launch only from here on
-      // chunk groups of this CTA: zk counts them; the set of group zk is zk & 1
+      bool failed = false;
       int zk = 0;
-      int cur_cg = nseg > 0 ? sg0.cg : -1;
-      const int last_cg = nseg > 0 ? seg_of(s1 - 1, p, C).cg : -1;
-      if (nseg > 0 && last_cg > cur_cg) {   // second group: produce it now
-        const Seg sg2 = seg_of((cur_cg + 1) * p.RT, p, C);
-        load_set_inputs<B>(p, vscr, xscr, sg2, tid);
-        named_sync(kBarEpi, 128);
-        produce_set<B, 128>(sets + K::SET, vscr, xscr, xsf, p.x_bf16, ctl, sg2, tid, kBarEpi, &ctl->zfull[1], false);
-      }
-      uint32_t zr[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) zr[q] = 0u;
-      for (int j = 0; j < nseg; ++j) {
-        const Seg sg = seg_of(s0 + j, p, C);
-        if (sg.cg != cur_cg) {
-          cur_cg = sg.cg;
-          ++zk;
-        }
-        const float* hdr = reinterpret_cast<const float*>(sets + (zk & 1) * K::SET);
-        const int acc = j & 1;
-        const int us = j % kURing;
-        // this row's U_i entries (16 fp16), from the U ring
-        if (!failed) check(mbar_wait(&ctl->ufull[us], static_cast<uint32_t>((j / kURing) & 1), deadline, abort_flag));
-        uint4 ua = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
-        if (!failed) {
-          ua = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32);
-          ub = *reinterpret_cast<const uint4*>(uring + us * kTileBytes + tid * 32 + 16);
-        }
-        if (!failed) check(mbar_wait(&ctl->accfull[acc], static_cast<uint32_t>((j >> 1) & 1), deadline, abort_flag));
-        if (!failed) {
+      Seg sg = sg0;
+      for (int j = 0; j < nseg; ++j, seg_next(sg, p, C)) {
+        const int a = j % NACC;
+        const uint4* urow = reinterpret_cast<const uint4*>(record(p, sg.i) + u_offset(p) +
+                                                           static_cast<size_t>(sg.rt * kTileRows + tid) * kK * 2);
+        const uint4 ua = __ldg(urow), ub = __ldg(urow + 1);
+        bool ok = !failed && mbar_wait(&ctl->accfull[a], static_cast<uint32_t>((j / NACC) & 1), deadline, abort_flag);
+        ok = __all_sync(FULL, ok);
+        if (ok) {
           tc_fence_after();
+          const float* sig = ctl->sig[zk & 1];
+          const int* cs = ctl->csum[zk & 1];
           const __half* uh = reinterpret_cast<const __half*>(&ua);
           const __half* uh2 = reinterpret_cast<const __half*>(&ub);
-          const uint32_t abase = tmem + lane_base + static_cast<uint32_t>(acc * NB);
+          const uint32_t abase = tmem + lane_base + static_cast<uint32_t>(a * NB);
           float part[B];
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             uint32_t vh[16], vl[16];
             tmem_ld16(abase + b * 16, vh);
-            tmem_ld16(abase + 16 * B + b * 16, vl);
+            tmem_ld16(abase + NCOL + b * 16, vl);
             tc_wait_ld();
-            float sacc = 0.0f;
+            float acc = 0.0f;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-              const float slo = hdr[b * 16 + jj];
-              const float sbz = 256.0f * slo * static_cast<float>(static_cast<int>(vh[jj])) +
-                                slo * static_cast<float>(static_cast<int>(vl[jj]));
-              // S = 1 - 2 Sb (bit 1 = sign -1):  T = sum_c Z - 2 sum_c Sb Z
-              const float tval = hdr[64 + b * 16 + jj] - 2.0f * sbz;
+              const int col = b * 16 + jj;
+              // the accumulators hold -128 sum_c Sb hi and -128 sum_c Sb lo (exact
+              // multiples); S = 1 - 2 Sb:  T / sigma = sum_c q - 2 sum_c Sb q, in int32
+              const int sh = -static_cast<int>(vh[jj]) >> 7, sl = -static_cast<int>(vl[jj]) >> 7;
+              const int tq = cs[col] - 2 * (256 * sh + sl);
               const float uj = __half2float(jj < 8 ? uh[jj] : uh2[jj - 8]);
-              sacc = fmaf(uj, tval, sacc);
+              acc = fmaf(__fmul_rn(uj, sig[col]), static_cast<float>(tq), acc);
             }
-            part[b] = sacc;
+            part[b] = acc;
           }
-          // zero the accumulator for segment j + 2 and hand it back to the issuers
+          // zero the accumulator for the segment NACC later and hand it back
 #pragma unroll
           for (int cc = 0; cc < NB; cc += 32) tmem_st32(abase + cc, zr);
           tc_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) red_release_shared_add(&ctl->acc_free[acc], 1u);
+          if (lane == 0) mbar_arrive(&ctl->acc_free[a]);
           float* dst = p.part + static_cast<size_t>(s0 + j) * B * kTileRows;
 #pragma unroll
           for (int b = 0; b < B; ++b) dst[b * kTileRows + tid] = part[b];
+        } else {
+          set_error(p, ctl);
+          failed = true;   // keep walking: every warp must pass the same barriers below
         }
-        // U slot us is read by every epilogue thread: refill it for segment j + kURing
-        named_sync(kBarEpi, 128);
-        if (tid == 0 && j + kURing < nseg) {
-          const Seg sn = seg_of(s0 + j + kURing, p, C);
-          mbar_arrive_expect_tx(&ctl->ufull[us], kTileBytes);
-          bulk_g2s(uring + us * kTileBytes, u_tile(p, sn.i, sn.rt), kTileBytes, &ctl->ufull[us]);
-        }
-        // The last segment of group zk is done: its MMAs have completed, so the set of
-        // zk can take group zk + 2 if this CTA has one.
-        const bool group_end = (j + 1 == nseg) || seg_of(s0 + j + 1, p, C).cg != cur_cg;
-        if (group_end && cur_cg + 2 <= last_cg) {
-          const Seg sg3 = seg_of((cur_cg + 2) * p.RT, p, C);
-          load_set_inputs<B>(p, vscr, xscr, sg3, tid);
-          named_sync(kBarEpi, 128);
-          produce_set<B, 128>(sets + (zk & 1) * K::SET, vscr, xscr, xsf, p.x_bf16, ctl, sg3, tid, kBarEpi,
-                              &ctl->zfull[zk & 1], false);
+        const bool group_end = (j + 1 == nseg) || sg.rt + 1 == p.RT;
+        if (group_end) {
+          // this group's set and its sig / csum are no longer read: build group zk + 2
+          // (if the CTA has one) into the same slot
+          if (bar_any(kBarEpi, 128, failed || *abort_flag != 0)) {
+            failed = true;
+          } else if (zk + 2 < NZ) {
+            build_set_global<B>(p, ctl, zk & 1, sets + (zk & 1) * K::SET, sg.cg + 2, et, 128, kBarEpi);
+            if (et == 0) mbar_arrive(&ctl->zready[zk & 1]);
+          }
+          ++zk;
         }
       }
-      if (failed) set_error(p, ctl);
-
-      // ------------- row tiles: count the segments, then reduce the owned row tiles ---
-      // Row tile rt is reduced by CTA rt mod grid once all NC partials have arrived:
-      // fixed chunk-group order, so the sum is deterministic.
-      __threadfence();
-      named_sync(kBarEpi, 128);
-      if (tid == 0) ctl->abort_snap = *abort_flag;
-      named_sync(kBarEpi, 128);
-      if (!ctl->abort_snap) {
-        for (int e = tid; e < nseg; e += 128) atomicAdd(p.cnt + seg_of(s0 + e, p, C).rt, 1u);
-        const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
-        for (int rt = cta; rt < p.RT; rt += grid) {
-          if (tid == 0) {
-            bool ok = true;
-            while (ld_acquire_u32(p.cnt + rt) != static_cast<uint32_t>(NC)) {
-              if (*abort_flag || globaltimer_ns() > deadline) {
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-            ctl->red_ok = ok ? 1 : 0;
-            if (!ok) set_error(p, ctl);
-          }
-          named_sync(kBarEpi, 128);
-          if (ctl->red_ok) {
-            __threadfence();
-            const float* pp = p.part + static_cast<size_t>(rt) * B * kTileRows + tid;
-            constexpr int kBatch = 32 / B;   // loads in flight per thread
-            float acc[B];
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-            for (int c0 = 0; c0 < NC; c0 += kBatch) {
-              float v[kBatch][B];
-#pragma unroll
-              for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-                for (int b = 0; b < B; ++b)
-                  v[u][b] = c0 + u < NC ? __ldcg(pp + (c0 + u) * stride + b * kTileRows) : 0.0f;
-#pragma unroll
-              for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-                for (int b = 0; b < B; ++b) acc[b] += v[u][b];
-            }
-#pragma unroll
-            for (int b = 0; b < B; ++b)
-              store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + tid, acc[b]);
-            if (tid == 0) p.cnt[rt] = 0u;   // the next call starts from zero
-          }
-          named_sync(kBarEpi, 128);
-        }
-      }
-    } else if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuers -------
-      // Lane 0 of warp 8 + w issues K-steps w and w + 4 of every unit into the
-      // segment's accumulator (which the epilogue zeroes, so every MMA accumulates) and
-      // commits once per A-buffer pair and once per segment.  It waits for the
-      // expanders and the epilogue by polling shared counters: an mbarrier wait, or a
-      // whole warp walking the loop, costs the issuing thread more than its MMAs.
-      const int w = warp - kWarpIss0;
-      bool ok = !pfailed;
-      bool any = false;
-      int j = 0, c = 0, zk = -1, cur_cg = -1;
-      Seg sg = sg0;
-      uint32_t zbase = 0;
-      for (int g = 0; j < nseg && ok; ++g) {
-        const int pr = g % NPAIRS;
-        ok = poll_geq4(ctl->a_ready + 4 * (g & 1), static_cast<uint32_t>((g >> 1) + 1), deadline, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        for (int q = 0; q < kGroup && j < nseg && ok; ++q) {
-          const int acc = j & 1;
-          if (c == 0) {   // segment j starts: its accumulator must be zeroed
-            ok = poll_geq(&ctl->acc_free[acc], 4u * static_cast<uint32_t>((j >> 1) + 1), deadline, abort_flag);
-            tc_fence_after();
-            if (sg.cg != cur_cg) {
-              cur_cg = sg.cg;
-              ++zk;
-              if (ok) ok = mbar_wait(&ctl->zfull[zk & 1], static_cast<uint32_t>((zk >> 1) & 1), deadline, abort_flag);
-              zbase = smem_u32(sets + (zk & 1) * K::SET + kSetHdr);
-            }
-            if (!ok) break;
-          }
-          const uint32_t zaddr = zbase + static_cast<uint32_t>(c * K::ZB);
-          const uint32_t acol = K::ACOL0 + 64u * static_cast<uint32_t>(kGroup * pr + q);
-          const uint32_t dcol = static_cast<uint32_t>(acc * NB);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int t = w + kNI * h;
-            const uint64_t bdesc = smem_desc_noswizzle(zaddr + t * (NB / 8) * 256, 128, 256);
-            mma_i8_ts(tmem + dcol, tmem + acol + 8 * t, bdesc, IDESC, 1u);
-          }
-          any = true;
-          if (++c == sg.len) {
-            tc_commit(&ctl->accfull[acc]);
-            c = 0;
-            ++j;
-            if (j < nseg) sg = seg_of(s0 + j, p, C);
-          }
-        }
-        if (ok) tc_commit(&ctl->aempty[pr]);
-      }
-      if (!ok) set_error(p, ctl);
-      if (any) {
-        tc_commit(&ctl->drain[w]);
-        mbar_wait(&ctl->drain[w], 0, globaltimer_ns() + 100000000ull, nullptr);
-      }
+      __threadfence();   // this thread's partials are visible before any arrival is counted
+      const bool stop = bar_any(kBarEpi, 128, failed || *abort_flag != 0);
+      if (et == 0) ctl->count_ok = stop ? 0 : 1;
     }
-  } else if (warp == kWarpCopy && lane == 0) {
-    // ------------------------------------------------------ sign-tile copies -------
-    // Stack memory only (it may be read before the previous kernel in the stream has
-    // finished): V rows of the first chunk group, the first sign stages and U tiles.
-    int issued = 0;
-    if (nseg > 0) {
-      const uint32_t vb = static_cast<uint32_t>(sg0.len) * kTileCols * kK * 2;
-      mbar_arrive_expect_tx(&ctl->vfull, vb);
-      bulk_g2s(vscr, v_rows(p, sg0), vb, &ctl->vfull);
-    }
-    for (; issued < NS && issued < nseg; ++issued) {
-      if (p.inject_unreachable && issued == 0) continue;
-      const Seg sg = seg_of(s0 + issued, p, C);
-      const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
-      mbar_arrive_expect_tx(&ctl->sfull[issued], bytes);
-      bulk_g2s(stages + issued * K::STAGE,
-               p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
-                   (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
-               bytes, &ctl->sfull[issued]);
-    }
-    for (int j = 0; j < kURing && j < nseg; ++j) {
-      const Seg sg = seg_of(s0 + j, p, C);
-      mbar_arrive_expect_tx(&ctl->ufull[j], kTileBytes);
-      bulk_g2s(uring + j * kTileBytes, u_tile(p, sg.i, sg.rt), kTileBytes, &ctl->ufull[j]);
-    }
-    for (; issued < nseg; ++issued) {
-      const int st = issued % NS;
-      if (!mbar_wait(&ctl->sempty[st], static_cast<uint32_t>((issued / NS - 1) & 1), deadline, abort_flag)) {
-        set_error(p, ctl);
-        break;
-      }
-      const Seg sg = seg_of(s0 + issued, p, C);
-      const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
-      mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
-      bulk_g2s(stages + st * K::STAGE,
-               p.blocks + static_cast<size_t>(sg.i) * p.block_bytes +
-                   (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes,
-               bytes, &ctl->sfull[st]);
-    }
-    // No copy may be in flight when the CTA exits: wait for the last use of every
-    // stage and for the first-group inputs (each bounded).
-    const uint64_t drain_by = globaltimer_ns() + 100000000ull;
-    for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q) {
-      if (p.inject_unreachable && q == 0) continue;
-      mbar_wait(&ctl->sfull[q % NS], static_cast<uint32_t>((q / NS) & 1), drain_by, nullptr);
-    }
-    if (nseg > 0) mbar_wait(&ctl->vfull, 0, drain_by, nullptr);
   }
 
-  // U-ring copies are issued by epilogue thread 0 (and the copy thread): drain them too.
-  if (warp == kWarpEpi0 && lane == 0) {
-    const uint64_t drain_by = globaltimer_ns() + 100000000ull;
-    for (int j = (nseg > kURing ? nseg - kURing : 0); j < nseg; ++j)
-      mbar_wait(&ctl->ufull[j % kURing], static_cast<uint32_t>((j / kURing) & 1), drain_by, nullptr);
-  }
+  // --------------------------------------------------- row tiles: count and reduce -----
+  // Every warp of the CTA takes part.  The CTA counts its partials into the row tiles'
+  // arrival counters; the CTA that adds a tile's last partial sums all of them and
+  // writes y.  No CTA waits for another; a CTA that failed counts nothing.  The sum has
+  // a fixed association whichever CTA runs it: thread (row r, slice k) of the K =
+  // threads / 128 slices adds the partials of chunk groups k, k + K, ... in order, and
+  // the K slice sums are added in slice order.
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpCopy) {
+  if (ctl->count_ok) {
+    constexpr int KS = K::THREADS / kTileRows;   // slices per row tile
+    const int NC = p.n * p.NCB;                  // partials per row tile
+    const int r = threadIdx.x % kTileRows, ks = threadIdx.x / kTileRows;
+    // the sign stages are drained by now: [4 tiles][KS][B][128] slice sums, then the row
+    // tiles this CTA completed in the current round
+    float* red = reinterpret_cast<float*>(stages);
+    int* red_rt = reinterpret_cast<int*>(stages + 4 * KS * B * kTileRows * 4);
+    for (int base = 0; base < nseg; base += K::THREADS) {
+      const int e = base + static_cast<int>(threadIdx.x);
+      if (e < nseg) {
+        const int rt = (s0 + e) % p.RT;
+        if (atomicAdd(p.cnt + rt, 1u) == static_cast<uint32_t>(NC - 1)) {
+          const int idx = atomicAdd(&ctl->nred, 1);
+          red_rt[idx] = rt;
+        }
+      }
+      __syncthreads();
+      const int nred = ctl->nred;
+      if (nred > 0) __threadfence();
+      // up to kTB row tiles per pass, their loads all in flight together
+      constexpr int kTB = 4;
+      for (int q0 = 0; q0 < nred; q0 += kTB) {
+        const int nq = min(kTB, nred - q0);
+        if (ks < KS) {
+          const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
+          float acc[kTB][B];
+#pragma unroll
+          for (int t = 0; t < kTB; ++t)
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[t][b] = 0.0f;
+          for (int c0 = ks; c0 < NC; c0 += 4 * KS) {
+            float v[kTB][4][B];
+#pragma unroll
+            for (int t = 0; t < kTB; ++t) {
+              const float* pp = p.part + static_cast<size_t>(t < nq ? red_rt[q0 + t] : 0) * B * kTileRows + r;
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2)
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                  const int cg = c0 + e2 * KS;
+                  v[t][e2][b] = (t < nq && cg < NC) ? __ldcg(pp + cg * stride + b * kTileRows) : 0.0f;
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < kTB; ++t)
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2)
+#pragma unroll
+                for (int b = 0; b < B; ++b) acc[t][b] += v[t][e2][b];
+          }
+#pragma unroll
+          for (int t = 0; t < kTB; ++t)
+#pragma unroll
+            for (int b = 0; b < B; ++b) red[((t * KS + ks) * B + b) * kTileRows + r] = acc[t][b];
+        }
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < nq * kTileRows; idx += K::THREADS) {
+          const int t = idx / kTileRows, rr = idx - t * kTileRows;
+          const int rt = red_rt[q0 + t];
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            float sum = 0.0f;
+            for (int k = 0; k < KS; ++k) sum += red[((t * KS + k) * B + b) * kTileRows + rr];
+            store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + rr, sum);
+          }
+          if (rr == 0) p.cnt[rt] = 0u;   // the next call starts from zero
+        }
+        __syncthreads();
+      }
+      if (threadIdx.x == 0) ctl->nred = 0;
+      __syncthreads();
+    }
+  }
+
+  if (warp == K::WCTL) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -708,15 +850,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 
 template <int B>
 cudaError_t launch_b(const DecodeParams& p, int grid, cudaStream_t stream) {
+  using K = Cfg<B>;
   auto kern = decode_kernel<B>;
-  constexpr int smem = Cfg<B>::SMEM;
   static bool configured[64] = {};   // the attribute is set once per device, outside any capture
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
@@ -724,12 +866,12 @@ cudaError_t launch_b(const DecodeParams& p, int grid, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cfg.stream = stream;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(K::THREADS);
+  cfg.dynamicSmemBytes = K::SMEM;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

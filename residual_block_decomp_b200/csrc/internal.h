@@ -21,18 +21,23 @@ constexpr uint32_t kErrTimeout = 1u;   // device error word bit: a bounded wait 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Decode work unit: a segment = one 128-row tile x up to C consecutive 256-column
-// chunks of one block (C = decode_chunks_per_segment(batch)).  Segments are numbered
-// s = cg * RT + rt over chunk groups cg = i * NCB + (kg / C) of block i.
+// chunks of one block (C = decode_chunks_per_segment(batch)); the C chunks of a block
+// that share a segment form a chunk group.  Segments are numbered s = cg * RT + rt over
+// chunk groups cg = i * NCB + (kg / C) of block i.
 __host__ __device__ constexpr int decode_chunks_per_segment(int batch) { return batch == 1 ? 4 : 2; }
 inline int decode_groups_per_block(int d, int batch) {
   const int KG = d / kTileCols, C = decode_chunks_per_segment(batch);
   return (KG + C - 1) / C;
 }
+// Activation operand of one chunk group ("set"), built in shared memory by the decode
+// kernel: C chunks of the two int8 planes in the tensor-core operand layout (32 * batch
+// operand columns x 256 K-elements, one byte each).
+__host__ __device__ constexpr int decode_chunk_operand_bytes(int batch) { return 32 * batch * kTileCols; }
 
 // Decode workspace carve-up (256-byte aligned regions): one arrival counter per row
-// tile, then per-segment partial outputs.  The counters come first so that their
-// place does not move with n_loaded or batch: a workspace reused by calls with other
-// sizes still finds them at zero (every completed call leaves them at zero).
+// tile, then per-segment partial outputs.  The counters come first so that their place
+// does not move with n_loaded or batch: a workspace reused by calls with other sizes
+// still finds them at zero (every completed call leaves them at zero).
 struct DecodeWs {
   size_t cnt, part, total;
 };
@@ -54,12 +59,12 @@ struct DecodeParams {
   void* y;                     // batch x m, same dtype
   const float* inv_s;          // d
   float* part;                 // [segs][batch][128] partial outputs of the segments
-  uint32_t* cnt;               // [RT] segments of the row tile reduced so far
+  uint32_t* cnt;               // [RT] partials of the row tile that have arrived
   uint32_t* err;               // sticky device error word
   int m, d, n, KG, RT, NCB;    // NCB chunk groups per block
   int segs;                    // RT * n * NCB
   int x_bf16;
-  int inject_unreachable;      // the first sign copy of every CTA is never issued (timeout test)
+  int inject_unreachable;      // CTA 0's first sign copy is never issued (timeout test)
   unsigned long long timeout_ns;
 };
 
@@ -83,6 +88,11 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, cons
                            const CUtensorMap& tm_v, int bf16, cudaStream_t stream);
 size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs);
 
+// bs_linear_no_alloc keeps its scratch in one array per device, shared by every stack
+// on that device: an error reported on any stack marks the device's array for clearing
+// before the next no-alloc call there (no_alloc.cu).
+void note_device_error(int device);
+
 cudaError_t launch_reconstruct(const uint8_t* blocks, unsigned long long block_bytes, const float* inv_s, int m,
                                int d, int n, void* out, int dtype, cudaStream_t stream);
 cudaError_t launch_unpack(const uint8_t* record, int m, int d, int8_t* out, cudaStream_t stream);
@@ -99,7 +109,6 @@ struct bs_stack_s {
   int device, sm_count;
   unsigned long long timeout_ns;
   int inject_unreachable;
-  int scratch_dirty;       // an error was reported: bs_linear_no_alloc clears its scratch first
   CUtensorMap tm_u, tm_v;  // prefill operand maps over the whole block area
   int tmaps_ready;
 };

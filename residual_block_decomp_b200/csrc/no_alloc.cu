@@ -19,11 +19,13 @@
 // All calls on a device share the one array, and it keeps whatever the previous call
 // left in it; a decode call that completes leaves its row-tile counters at zero, so
 // no clearing is needed between calls.  A call that ran out of a bounded wait may
-// leave counters behind: once bs_get_device_error has reported an error on a stack,
-// the next call here on that stack clears the array first (an asynchronous memset on
-// the call's stream).  Two calls whose kernels may overlap on the GPU (different
-// streams, no ordering between them) race on the array: order them on one stream,
-// or give them distinct workspaces through bs_linear.
+// leave counters behind, and the array belongs to every stack on the device: once
+// bs_get_device_error has reported an error on any stack of a device, the next
+// no-alloc call on that device, whatever its stack, clears the whole array first (an
+// asynchronous memset on the call's stream).  Two calls whose kernels may overlap on
+// the GPU (different streams, no ordering between them) race on the array: order them
+// on one stream, or give them distinct workspaces through bs_linear.
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -36,6 +38,7 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 void* g_scratch_addr[kMaxDevices] = {};
+std::atomic<int> g_scratch_dirty[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
 // Device address of g_static_scratch on the current device; set up on first use.
@@ -47,12 +50,19 @@ bs_status scratch_address(int device, void** out) {
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return BS_ERR_CUDA;
     if (cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) return BS_ERR_CUDA;
     g_scratch_addr[device] = p;
+    g_scratch_dirty[device].store(0);
   }
   *out = g_scratch_addr[device];
   return BS_OK;
 }
 
 }  // namespace
+
+namespace bs {
+void note_device_error(int device) {
+  if (device >= 0 && device < kMaxDevices) g_scratch_dirty[device].store(1);
+}
+}  // namespace bs
 
 extern "C" bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded,
                                         void* y, bs_stream_t stream) {
@@ -67,9 +77,11 @@ extern "C" bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int bat
   void* scratch = nullptr;
   const bs_status st = scratch_address(device, &scratch);
   if (st != BS_OK) return st;
-  if (stack->scratch_dirty) {
-    if (cudaMemsetAsync(scratch, 0, need, stream) != cudaSuccess) return BS_ERR_CUDA;
-    stack->scratch_dirty = 0;
+  if (g_scratch_dirty[device].exchange(0) != 0) {
+    if (cudaMemsetAsync(scratch, 0, kStaticScratchBytes, stream) != cudaSuccess) {
+      g_scratch_dirty[device].store(1);
+      return BS_ERR_CUDA;
+    }
   }
   return bs_linear(stack, x, batch, dt, n_loaded, y, scratch, kStaticScratchBytes, stream);
 }

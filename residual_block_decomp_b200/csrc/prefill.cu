@@ -345,15 +345,20 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, cons
                            const CUtensorMap& tm_v, int bf16, cudaStream_t stream) {
   const size_t smem = prefill_smem_bytes(p.n, p.NT, p.xstages, p.sbufs);
   dim3 grid(p.m / kTileRows, (p.M + p.NT - 1) / p.NT);
-  static int configured[2] = {0, 0};  // set once per dtype (stream capture never sees it)
-  if (configured[bf16 ? 1 : 0] < static_cast<int>(smem)) {
-    const cudaError_t e =
-        bf16 ? cudaFuncSetAttribute(prefill_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // the attribute is per device and kernel: set it once for each (device, dtype), outside
+  // any stream capture (the first call on a device must not be captured)
+  static bool configured[64][2] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev][bf16 ? 1 : 0]) {
+    e = bf16 ? cudaFuncSetAttribute(prefill_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(227 * 1024))
              : cudaFuncSetAttribute(prefill_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(227 * 1024));
     if (e != cudaSuccess) return e;
-    configured[bf16 ? 1 : 0] = 227 * 1024;
+    configured[dev][bf16 ? 1 : 0] = true;
   }
   if (bf16) {
     prefill_kernel<__nv_bfloat16><<<grid, kThreads, smem, stream>>>(p, tm_x, tm_u, tm_v);

@@ -1,52 +1,82 @@
 """CPU: the decode kernel's work split and memory geometry, mirrored on the host.
 
 The decode kernel (csrc/decode.cu) cuts a call into segments (one 128-row tile of one
-block x C chunks of 256 columns, chunk-group-major) and gives each CTA a contiguous run.
-This test restates that arithmetic and checks, for the shapes the tests and the bench
-use, that
-  * every unit (row tile, block, chunk) is covered exactly once;
-  * every bulk copy (sign stage, V rows, U tile) lies inside its block's area;
+block x one chunk group, chunk-group-major), gives each CTA a contiguous run, builds
+the activation sets of its chunk groups in two shared-memory slots, streams each
+segment's sign tiles into shared-memory stages, hands units to teams of four warps and
+to the issuer warps in turn, and reduces each row tile in the CTA that adds its last
+partial.  This test restates that arithmetic and checks, for the shapes the tests and
+the bench use, that
+  * every unit (row tile, block, chunk) is covered exactly once, by exactly one team
+    and one issuer;
+  * every bulk copy (sign stage) and every V / U row read lies inside its source area;
   * a CTA touches consecutive chunk groups only;
-  * the per-CTA shared memory fits 227 KB and the tensor-memory columns fit 512;
+  * the activation-set bytes the builders write land exactly where the MMA descriptors
+    read them, and tile each chunk exactly;
+  * shared memory, tensor-memory columns and threads fit, and two decode CTAs never
+    share an SM;
+  * the per-segment barrier arrivals add up to the counts the barriers are set to;
   * the reduction reads stay inside the workspace that bs_workspace_bytes reports.
-A change to the kernel's split or layout that breaks one of these fails here, on the
+A change to the kernels' split or layout that breaks one of these fails here, on the
 CPU, before anything runs on a GPU."""
+import numpy as np
 import pytest
 
 import residual_block_decomp_b200 as R
 
-SMEM_LIMIT = 227 * 1024
+SM_SMEM = 228 * 1024
+RESERVED = 1024
+BLOCK_LIMIT = 227 * 1024
 SMS = 148
 
 
-def chunks_per_segment(b):
-    return 4 if b == 1 else 2
+class Cfg:
+    def __init__(self, b):
+        self.B = b
+        self.NB = 32 * b
+        self.NCOL = 16 * b
+        self.C = 4 if b == 1 else 2
+        self.ZB = self.NB * 256
+        self.SET = self.C * self.ZB
+        self.T = 3 if b <= 2 else 2
+        self.NI = 3
+        self.NACC = 4 if b == 1 else 2
+        self.ACOL0 = self.NACC * self.NB
+        self.THREADS = 32 * (4 * self.T + self.NI + 5)
+        self.ZTHREADS = self.THREADS - 32
+        self.STAGE = self.C * 4096
+        stg = b * self.C * 256 * 2 + self.C * 256 * 4          # first group's x rows and 1/s
+        self.STG_AL = -(-stg // 1024) * 1024
+        fixed = 2 * self.SET + 8192 + self.STG_AL
+        self.NS = min(16, (BLOCK_LIMIT - fixed) // self.STAGE)
+        self.SMEM = self.NS * self.STAGE + fixed
 
 
-def shared_memory(b):
-    """Bytes of dynamic shared memory per CTA: sign stages + two chunk-group sets +
-    V rows + x rows and 1/s + x (.) 1/s + U ring + control block."""
-    nb, C = 32 * b, chunks_per_segment(b)
-    cols = C * 256
-    fixed = 2 * (512 + C * nb * 256) + cols * 32 + (cols * b * 2 + cols * 4) + cols * b * 4 + 4 * 4096 + 1024
-    stage = C * 4096
-    ns = min(16, (SMEM_LIMIT - fixed) // stage)
-    return ns, ns * stage + fixed
-
-
-def tmem_columns(b):
-    nb = 32 * b
-    pairs = (512 - 2 * nb) // 128
-    return pairs, 2 * nb + 128 * pairs
+def cta_range(cta, grid, n, NCB, RT):
+    """Mirror of the kernel's cta_range: group-aligned runs when the chunk groups are no
+    more than the CTAs, contiguous runs otherwise."""
+    NG, segs = n * NCB, RT * n * NCB
+    if NG <= grid:
+        base, extra = divmod(grid, NG)
+        if cta < extra * (base + 1):
+            g, w = divmod(cta, base + 1)
+            k = base + 1
+        else:
+            c2 = cta - extra * (base + 1)
+            g = extra + c2 // base
+            w = c2 - (g - extra) * base
+            k = base
+        return g * RT + (w * RT) // k, g * RT + ((w + 1) * RT) // k
+    return cta * segs // grid, (cta + 1) * segs // grid
 
 
 def geometry(m, d, n, b):
-    C = chunks_per_segment(b)
+    K = Cfg(b)
     RT, KG = m // 128, d // 256
-    NCB = -(-KG // C)
+    NCB = -(-KG // K.C)
     segs = RT * n * NCB
-    grid = min(SMS, segs)
-    return C, RT, KG, NCB, segs, grid
+    grid = min(SMS - 4, segs)
+    return K, RT, KG, NCB, segs, grid
 
 
 SHAPES = [(128, 256, 1), (256, 512, 3), (384, 768, 2), (640, 1280, 4), (1024, 4096, 5), (512, 2560, 7),
@@ -54,46 +84,104 @@ SHAPES = [(128, 256, 1), (256, 512, 3), (384, 768, 2), (640, 1280, 4), (1024, 40
 
 
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
-def test_shared_and_tensor_memory_fit(b):
-    ns, smem = shared_memory(b)
-    assert ns >= 2 and smem <= SMEM_LIMIT
-    pairs, cols = tmem_columns(b)
-    assert 2 <= pairs <= 3 and cols <= 512
+def test_shared_tensor_memory_and_threads_fit(b):
+    K = Cfg(b)
+    assert K.NS >= 4 and K.SMEM <= BLOCK_LIMIT
+    # two decode CTAs (each allocating all 512 tensor-memory columns) never share an SM
+    assert 2 * (K.SMEM + RESERVED) > SM_SMEM
+    assert K.ACOL0 + K.T * 2 * 64 <= 512
+    assert K.THREADS <= 1024
+    # the epilogue warps start at 4T + NI: with the issuers in between, their indices
+    # modulo 4 still cover the four tensor-memory lane quadrants once each
+    wepi = 4 * K.T + K.NI
+    assert sorted(w % 4 for w in range(wepi, wepi + 4)) == [0, 1, 2, 3]
+    # the activation sets sit at the start of shared memory: descriptor addresses fit
+    # their 14-bit field (16-byte units)
+    assert (2 * K.SET) >> 4 < (1 << 14)
+    # the first group's V rows (32 bytes per input column) are staged in the second set
+    # slot, its x rows and 1/s in the staging area
+    assert K.C * 256 * 32 <= K.SET
+    assert b * K.C * 256 * 2 + K.C * 256 * 4 <= K.STG_AL
 
 
 @pytest.mark.parametrize("m,d,n", SHAPES)
 @pytest.mark.parametrize("b", [1, 4])
 def test_segments_cover_units_once_and_stay_in_bounds(m, d, n, b):
-    C, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
+    K, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
     sign_bytes = m * d // 8
     seen = set()
+    groups = n * NCB
     for cta in range(grid):
-        s0, s1 = cta * segs // grid, (cta + 1) * segs // grid
+        s0, s1 = cta_range(cta, grid, n, NCB, RT)
         assert s1 > s0
+        if groups <= grid:
+            assert s0 // RT == (s1 - 1) // RT       # inside one chunk group
         cgs = []
+        u = 0
         for s in range(s0, s1):
             cg, rt = divmod(s, RT)
             i, cgi = divmod(cg, NCB)
-            kgA = cgi * C
-            ln = min(C, KG - kgA)
-            assert 0 <= i < n and 1 <= ln <= C
+            kgA = cgi * K.C
+            ln = min(K.C, KG - kgA)
+            assert 0 <= i < n and 1 <= ln <= K.C
             # sign stage: ln contiguous 4 KiB tiles of row tile rt, inside block i's signs
-            assert (rt * KG + kgA) * 4096 + ln * 4096 <= sign_bytes
-            # V rows of the group and the row tile's U rows, inside the factor areas
-            assert (kgA * 256 + ln * 256) * 32 <= d * 32 and rt * 128 * 32 + 4096 <= m * 32
+            assert (rt * KG + kgA) * 4096 + ln * 4096 <= sign_bytes and ln * 4096 <= K.STAGE
+            # the group's V rows and the row tile's U rows inside the factor areas
+            assert (kgA * 256 + ln * 256) * 32 <= d * 32
+            assert (rt * 128 + 127) * 32 + 32 <= m * 32
             for kg in range(kgA, kgA + ln):
                 key = (rt, i, kg)
                 assert key not in seen
-                seen.add(key)
+                seen.add((rt, i, kg))
+                # unit u: team u mod T, slot (u // T) mod 2, issuer u mod NI
+                assert 0 <= u % K.T < K.T and 0 <= u % K.NI < K.NI
+                u += 1
             cgs.append(cg)
         assert sorted(set(cgs)) == list(range(cgs[0], cgs[-1] + 1))
     assert len(seen) == RT * n * KG
 
 
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_set_bytes_land_where_the_mma_reads(b):
+    """The set builders write the byte of operand column n (hi plane n = 16 b + j, lo
+    plane NCOL + n) and group column c at chunk c >> 8, K-step t = (c & 255) >> 5,
+    K-half kc = (c >> 4) & 1, byte c & 15 of the 16-byte row of core matrix (n >> 3,
+    kc), row n & 7.  The decode kernel's descriptor for K-step t (no swizzle, K-major,
+    LBO 128 = next core matrix in K, SBO 256 = next core matrix in N) reads that core
+    matrix row at t*(NB/8)*256 + (n>>3)*256 + kc*128 + (n&7)*16.  Both must agree, and
+    the writes must tile every chunk exactly once."""
+    K = Cfg(b)
+    hits = np.zeros(K.SET, dtype=np.int32)
+    for c in range(K.C * 256):
+        cc, cl = c >> 8, c & 255
+        t, kc, byte = cl >> 5, (cl >> 4) & 1, cl & 15
+        for n in range(K.NB):
+            written = cc * K.ZB + (t * (K.NB // 8) * 2 + kc) * 128 + byte + (n >> 3) * 256 + (n & 7) * 16
+            read = cc * K.ZB + t * (K.NB // 8) * 256 + (n >> 3) * 256 + kc * 128 + (n & 7) * 16 + byte
+            assert written == read
+            hits[written] += 1
+    assert hits.min() == 1 and hits.max() == 1
+
+
 @pytest.mark.parametrize("m,d,n", SHAPES)
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
-def test_reduction_reads_inside_workspace(m, d, n, b):
-    C, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
+def test_barrier_arrivals_match_counts(m, d, n, b):
+    """Per segment the issuer of each unit commits once into the segment's accumulator
+    barrier, and the issuer of a short segment's last unit adds C - len plain
+    arrivals; each of the four warps of a unit's team arrives once on the sign stage,
+    and adds C - len after the segment's last unit.  Every phase therefore receives the
+    count its barrier is set to (C and 4 C), short segments included."""
+    K, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
+    for cgi in range(NCB):
+        ln = min(K.C, KG - cgi * K.C)
+        assert ln + (K.C - ln) == K.C
+        assert 4 * ln + 4 * (K.C - ln) == 4 * K.C
+
+
+@pytest.mark.parametrize("m,d,n", SHAPES)
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_workspace_layout_and_reduction_reads(m, d, n, b):
+    K, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
     NC = n * NCB
     cnt_bytes = -(-RT * 4 // 256) * 256
     part_floats = segs * b * 128
@@ -109,7 +197,6 @@ def test_expansion_rule_reads_columns_in_order():
     2048 + r*16 (eight 32-bit words w[0..7]), and K-step t takes byte q of
     (w[pw] >> t) & 0x01010101 as A[r, 32 t + 4 pw + q].  Applied to the library's own
     host packer, that rule must give the signs in natural column order."""
-    import numpy as np
     gen = np.random.default_rng(11)
     m, d = 256, 512
     neg = gen.random((m, d)) < 0.5
