@@ -481,47 +481,47 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == K::WCTL) {
-    // ------------------------------------------------------------- copy thread -------
-    if (lane == 0) {
-      Seg sc = sg0;   // the segment of the next stage to issue (stages are issued in order)
-      auto issue_stage = [&](int jj) {
-        const Seg sg = sc;
-        seg_next(sc, p, C);
-        const int st = jj % NS;
-        const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
-        mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
-        bulk_g2s(stages + st * K::STAGE,
-                 record(p, sg.i) + (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes, bytes, &ctl->sfull[st]);
-      };
-      // The first group's V rows (into the second set slot) and 1/s, then the sign tiles:
-      // stack memory and the scale vector, read before the previous kernel has finished.
-      // (Timeout test: CTA 0 leaves out its first stage, so its waits run out while the
-      // other CTAs complete and count their partials.)
-      const Group G0 = group_of(p, sg0.cg, C);
+    // ------------------------------------------------------------- copy warp ---------
+    // Issuing a bulk copy costs the issuing thread a few hundred cycles, so the first
+    // stages (and the first group's inputs) are issued by the lanes in parallel, one copy
+    // each; later stages, which wait for freed slots, by lane 0.
+    const bool skip_first = p.inject_unreachable && cta == 0;   // timeout test: see below
+    auto issue_stage = [&](int jj, const Seg& sg) {
+      const int st = jj % NS;
+      const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
+      mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
+      bulk_g2s(stages + st * K::STAGE,
+               record(p, sg.i) + (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes, bytes, &ctl->sfull[st]);
+    };
+    // The first group's V rows (into the second set slot) and 1/s, and the first stages:
+    // stack memory and the scale vector, read before the previous kernel has finished.
+    // (Timeout test: CTA 0 leaves out its first stage, so its waits run out while the
+    // other CTAs complete and count their partials.)
+    const Group G0 = group_of(p, sg0.cg, C);
+    const int first = min(NS, nseg);
+    if (lane == 31) {
       mbar_arrive_expect_tx(&ctl->vstage, static_cast<uint32_t>(G0.gcols) * 36u);
       bulk_g2s(sets + K::SET, record(p, G0.i) + v_offset(p) + static_cast<size_t>(G0.col0) * 32,
                static_cast<uint32_t>(G0.gcols) * 32u, &ctl->vstage);
       bulk_g2s(stg + B * C * kTileCols * 2, p.inv_s + G0.col0, static_cast<uint32_t>(G0.gcols) * 4u, &ctl->vstage);
-      const bool skip_first = p.inject_unreachable && cta == 0;
-      int issued = 0;
-      for (; issued < NS && issued < nseg; ++issued) {
-        if (skip_first && issued == 0) {
-          seg_next(sc, p, C);
-          continue;
-        }
-        issue_stage(issued);
-      }
-      // x only after the kernel ahead has finished (it may have written x)
-      griddep_wait();
-      mbar_arrive_expect_tx(&ctl->xstage, static_cast<uint32_t>(B * G0.gcols) * 2u);
-      for (int b = 0; b < B; ++b)
-        bulk_g2s(stg + b * C * kTileCols * 2, static_cast<const uint16_t*>(p.x) + static_cast<size_t>(b) * p.d + G0.col0,
-                 static_cast<uint32_t>(G0.gcols) * 2u, &ctl->xstage);
+    }
+    if (lane < first && !(skip_first && lane == 0)) issue_stage(lane, seg_of(s0 + lane, p, C));
+    // x only after the kernel ahead has finished (it may have written x)
+    griddep_wait();
+    if (lane == 0) mbar_arrive_expect_tx(&ctl->xstage, static_cast<uint32_t>(B * G0.gcols) * 2u);
+    __syncwarp();
+    if (lane < B)
+      bulk_g2s(stg + lane * C * kTileCols * 2, static_cast<const uint16_t*>(p.x) + static_cast<size_t>(lane) * p.d + G0.col0,
+               static_cast<uint32_t>(G0.gcols) * 2u, &ctl->xstage);
+    if (lane == 0) {
+      Seg sc = seg_of(s0 + first, p, C);   // the segment of the next stage to issue
+      int issued = first;
       bool ok = true;
-      for (; ok && issued < nseg; ++issued) {
+      for (; issued < nseg; ++issued) {
         ok = mbar_wait(&ctl->sempty[issued % NS], static_cast<uint32_t>((issued / NS - 1) & 1), deadline, abort_flag);
-        if (ok) issue_stage(issued);
-        else break;
+        if (!ok) break;
+        issue_stage(issued, sc);
+        seg_next(sc, p, C);
       }
       if (!ok) set_error(p, ctl);
       // no copy may still be landing in shared memory when the CTA exits

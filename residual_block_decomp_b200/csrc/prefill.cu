@@ -8,15 +8,17 @@
 // so each CTA rebuilds tiles of W_hat on chip and never writes them to device memory:
 //
 //   for each 32-column K-tile of its 128 output rows:
-//     P_i = U_i[rows] V_i[cols]^T          rank-16 tcgen05 MMA (fp16) -> TMEM, per block
+//     P_i = U_i[rows] V_i[cols]^T          rank-16 tcgen05 MMA (fp16) -> TMEM, per block,
+//                                          four blocks per round, two rounds in flight
 //     W_t = (sum_i sign_i (.) P_i) / s     TMEM -> registers, sign applied by XOR
 //     W_t -> fp16/bf16 -> shared memory    the A operand of the GEMM
 //     y_tile += W_t x_tile^T               tcgen05 MMA, M = 128 rows, N = NT tokens
 //
 // Operands arrive by TMA (x tiles, U and V tiles; no multicast) and 1-D bulk copies
-// (sign tiles).  Warp roles: warps 0-3 rebuild and write the epilogue (thread = row =
-// TMEM lane), warp 4 issues copies, warp 5 owns TMEM and issues MMAs.  All waits are
-// bounded; a wait that runs out sets the device error word and the CTA unwinds.
+// (sign tiles).  Warp roles: warps 0-7 rebuild (two warps per TMEM lane quadrant, each
+// taking half of a K-tile's columns; thread = row = TMEM lane) and write the epilogue,
+// warp 8 issues copies, warp 9 owns TMEM and issues MMAs.  All waits are bounded; a
+// wait that runs out sets the device error word and the CTA unwinds.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -26,21 +28,20 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kWarpLoad = 4, kWarpMma = 5;
+constexpr int kThreads = 320;
+constexpr int kWarpLoad = 8, kWarpMma = 9;    // warps 0-7 rebuild (two per TMEM lane quadrant)
+constexpr int kRb = 256;                      // rebuild threads
 constexpr int kKT = 32;              // K columns per tile
-constexpr int kPRound = 8;           // blocks whose P tiles fit TMEM at once
-constexpr uint32_t kPcol = 256;      // TMEM column of the P region (acc at 0..NT)
-constexpr int kBarRb = 1;
+constexpr int kPRound = 4;           // blocks per P round (one TMEM region of 128 columns)
+constexpr uint32_t kPcol = 256;      // TMEM columns of the two P regions (acc at 0..NT)
 
 struct Ctl {
-  uint64_t ubar, pfull, pempty, accfull, drain;
+  uint64_t ubar, accfull, drain;
+  uint64_t pfull[2], pempty[2];      // P regions: products ready / read by the rebuild warps
   uint64_t wfull[2], wempty[2];
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ void rb_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarRb), "n"(128) : "memory"); }
 
 template <typename DT>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi);
@@ -107,12 +108,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->ubar, 1);
-    mbar_init(&ctl->pfull, 1);
-    mbar_init(&ctl->pempty, 128);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&ctl->pfull[g], 1);
+      mbar_init(&ctl->pempty[g], kRb);
+    }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&ctl->wfull[w], 128);
+      mbar_init(&ctl->wfull[w], kRb);
       mbar_init(&ctl->wempty[w], 1);
     }
     for (int s = 0; s < XS; ++s) {
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < SB; ++s) {
       mbar_init(&sgfull[s], 1);
-      mbar_init(&sgempty[s], 128);
+      mbar_init(&sgempty[s], kRb);
     }
     ctl->abort = 0;
     fence_barrier_init();
@@ -134,45 +137,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpLoad) {
     // ----------------------------------------------------------------- loader -----
+    // The whole warp walks the K-tiles; lane 0 waits for free stages and sets the byte
+    // counts, then the lanes issue one copy each: issuing a copy costs the issuing
+    // thread a few hundred cycles, so spreading a K-tile's 2 n + 4 tensor copies (and a
+    // group's n sign copies) over the lanes keeps the loads ahead of the MMAs.
+    const uint32_t FULL = 0xffffffffu;
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_u);
       prefetch_tmap(&tm_v);
-      bool ok = true;
       mbar_arrive_expect_tx(&ctl->ubar, static_cast<uint32_t>(n) * 4096u);
-      for (int i = 0; i < n; ++i) {
-        tma_load_3d(smem + L.u_off + i * 4096, &tm_u, 0, rt * kTileRows, i, &ctl->ubar);
-        tma_load_3d(smem + L.u_off + i * 4096 + 2048, &tm_u, 8, rt * kTileRows, i, &ctl->ubar);
+    }
+    __syncwarp();
+    for (int e = lane; e < 2 * n; e += 32)
+      tma_load_3d(smem + L.u_off + (e >> 1) * 4096 + (e & 1) * 2048, &tm_u, 8 * (e & 1), rt * kTileRows, e >> 1,
+                  &ctl->ubar);
+    bool ok = true;
+    int kt = 0;
+    for (; kt < KT && ok; ++kt) {
+      if (kt % 8 == 0) {
+        const int grp = kt / 8, sb = grp % SB, use = grp / SB;
+        if (lane == 0) {
+          if (use > 0) ok = mbar_wait(&sgempty[sb], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&sgfull[sb], static_cast<uint32_t>(n) * kTileBytes);
+        }
+        ok = __shfl_sync(FULL, ok, 0);
+        if (!ok) break;
+        for (int i = lane; i < n; i += 32) {
+          const uint8_t* src = p.blocks + static_cast<size_t>(i) * p.block_bytes +
+                               (static_cast<size_t>(rt) * p.KG + grp) * kTileBytes;
+          bulk_g2s(smem + L.s_off + sb * L.s_stride + i * kTileBytes, src, kTileBytes, &sgfull[sb]);
+        }
       }
-      int kt = 0;
-      for (; kt < KT && ok; ++kt) {
-        if (kt % 8 == 0) {
-          const int grp = kt / 8, sb = grp % SB, use = grp / SB;
-          if (use > 0 && !mbar_wait(&sgempty[sb], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&sgfull[sb], static_cast<uint32_t>(n) * kTileBytes);
-          for (int i = 0; i < n; ++i) {
-            const uint8_t* src = p.blocks + static_cast<size_t>(i) * p.block_bytes +
-                                 (static_cast<size_t>(rt) * p.KG + grp) * kTileBytes;
-            bulk_g2s(smem + L.s_off + sb * L.s_stride + i * kTileBytes, src, kTileBytes, &sgfull[sb]);
-          }
-        }
-        const int s = kt % XS, use = kt / XS;
-        if (use > 0 && !mbar_wait(&xempty[s], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&xfull[s], static_cast<uint32_t>(n) * 1024u + static_cast<uint32_t>(NT) * kKT * 2u);
-        uint8_t* vb = smem + L.v_off + s * L.v_stride;
-        for (int i = 0; i < n; ++i) {
-          tma_load_3d(vb + i * 1024, &tm_v, 0, kt * kKT, i, &xfull[s]);
-          tma_load_3d(vb + i * 1024 + 512, &tm_v, 8, kt * kKT, i, &xfull[s]);
-        }
-        uint8_t* xb = smem + L.x_off + s * L.x_stride;
-        for (int kc = 0; kc < 4; ++kc) tma_load_2d(xb + kc * NT * 16, &tm_x, kt * kKT + 8 * kc, tok0, &xfull[s]);
+      const int s = kt % XS, use = kt / XS;
+      if (lane == 0) {
+        if (use > 0) ok = mbar_wait(&xempty[s], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
+        if (ok) mbar_arrive_expect_tx(&xfull[s], static_cast<uint32_t>(n) * 1024u + static_cast<uint32_t>(NT) * kKT * 2u);
       }
+      ok = __shfl_sync(FULL, ok, 0);
+      if (!ok) break;
+      uint8_t* vb = smem + L.v_off + s * L.v_stride;
+      uint8_t* xb = smem + L.x_off + s * L.x_stride;
+      for (int e = lane; e < 2 * n + 4; e += 32) {
+        if (e < 2 * n) tma_load_3d(vb + (e >> 1) * 1024 + (e & 1) * 512, &tm_v, 8 * (e & 1), kt * kKT, e >> 1, &xfull[s]);
+        else tma_load_2d(xb + (e - 2 * n) * NT * 16, &tm_x, kt * kKT + 8 * (e - 2 * n), tok0, &xfull[s]);
+      }
+    }
+    if (lane == 0) {
       if (!ok) {
         ctl->abort = 1;
         atomicOr(p.err, kErrTimeout);
@@ -193,45 +204,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_g = make_idesc(1u, is_bf16, is_bf16, 128u, static_cast<uint32_t>(NT));
       bool ok = mbar_wait(&ctl->ubar, 0, deadline, abort_flag);
       bool issued_any = false;
-      int prounds = 0;  // P rounds issued so far (parity of pfull / pempty)
-      for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % XS;
-        const int w = kt & 1;
-        if (!mbar_wait(&xfull[s], static_cast<uint32_t>((kt / XS) & 1), deadline, abort_flag)) { ok = false; break; }
-        const uint32_t vaddr = smem_u32(smem + L.v_off + s * L.v_stride);
-        const uint32_t uaddr = smem_u32(smem + L.u_off);
-        for (int r = 0; r < rounds && ok; ++r) {
-          if (prounds > 0 &&
-              !mbar_wait(&ctl->pempty, static_cast<uint32_t>((prounds - 1) & 1), deadline, abort_flag)) {
-            ok = false;
-            break;
+      // Two streams from one thread: P rounds (rank-16 products of kPRound blocks into the
+      // two TMEM regions, as far ahead as a free region and a loaded V stage allow) and
+      // the GEMM of each K-tile once its W_hat tile is in shared memory.  Non-blocking
+      // barrier tests decide which goes next, so the products of the next rounds are
+      // computed while the rebuild warps read the current ones.
+      const int PR = KT * rounds;
+      int pr = 0, kg = 0;
+      const uint32_t uaddr = smem_u32(smem + L.u_off);
+      for (uint32_t spins = 0; ok && kg < KT;) {
+        bool progressed = false;
+        if (pr < PR) {
+          const int ktp = pr / rounds, r = pr - ktp * rounds, s = ktp % XS, g = pr & 1;
+          if (mbar_test(&xfull[s], static_cast<uint32_t>((ktp / XS) & 1)) &&
+              (pr < 2 || mbar_test(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1)))) {
+            tc_fence_after();
+            const uint32_t vaddr = smem_u32(smem + L.v_off + s * L.v_stride);
+            const int i1 = min(n, (r + 1) * kPRound);
+            for (int i = r * kPRound; i < i1; ++i) {
+              const uint64_t adesc = smem_desc_noswizzle(uaddr + i * 4096, 2048, 128);
+              const uint64_t bdesc = smem_desc_noswizzle(vaddr + i * 1024, 512, 128);
+              mma_f16_ss(tmem + kPcol + 128u * g + (i - r * kPRound) * 32, adesc, bdesc, idesc_p, 0u);
+            }
+            issued_any = true;
+            tc_commit(&ctl->pfull[g]);
+            ++pr;
+            progressed = true;
           }
+        }
+        const int w = kg & 1;
+        if (kg * rounds < pr && mbar_test(&ctl->wfull[w], static_cast<uint32_t>((kg >> 1) & 1))) {
           tc_fence_after();
-          const int i1 = min(n, (r + 1) * kPRound);
-          for (int i = r * kPRound; i < i1; ++i) {
-            const uint64_t adesc = smem_desc_noswizzle(uaddr + i * 4096, 2048, 128);
-            const uint64_t bdesc = smem_desc_noswizzle(vaddr + i * 1024, 512, 128);
-            mma_f16_ss(tmem + kPcol + (i - r * kPRound) * 32, adesc, bdesc, idesc_p, 0u);
+          const int s = kg % XS;
+          const uint32_t waddr = smem_u32(smem + L.w_off + w * kTileRows * kKT * 2);
+          const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
+            const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
+            mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
           }
-          issued_any = true;
-          tc_commit(&ctl->pfull);
-          ++prounds;
+          tc_commit(&ctl->wempty[w]);
+          tc_commit(&xempty[s]);   // the stage's V rows (read by this K-tile's P rounds) and x tile
+          ++kg;
+          progressed = true;
         }
-        if (!ok) break;
-        if (!mbar_wait(&ctl->wfull[w], static_cast<uint32_t>((kt >> 1) & 1), deadline, abort_flag)) {
-          ok = false;
-          break;
+        if (progressed) {
+          spins = 0;
+        } else if ((++spins & 63u) == 0u) {
+          if (*abort_flag || globaltimer_ns() > deadline) ok = false;
+          __nanosleep(20);
         }
-        tc_fence_after();
-        const uint32_t waddr = smem_u32(smem + L.w_off + w * kTileRows * kKT * 2);
-        const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
-          const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
-          mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kt > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&ctl->wempty[w]);
-        tc_commit(&xempty[s]);
       }
       if (ok) {
         tc_commit(&ctl->accfull);
@@ -245,9 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------ warps 0-3: rebuild, epilogue -------
-    const int tid = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ---------------------- warps 0-7: rebuild (half a K-tile each), epilogue -------
+    const int half = warp >> 2;                          // K-tile columns 16 half .. 16 half + 15
+    const int tid = (warp & 3) * 32 + lane;              // row of the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool failed = false;
     auto check = [&](bool ok) {
       if (!__all_sync(0xffffffffu, ok)) failed = true;
@@ -257,60 +280,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int grp = kt / 8, t = kt % 8, sb = grp % SB;
       const int w = kt & 1;
       if (t == 0 && !failed) check(mbar_wait(&sgfull[sb], static_cast<uint32_t>((grp / SB) & 1), deadline, abort_flag));
-      float acc[32];
+      // column c of the K-tile is bit 8 (c % 4) + t of word c / 4 of the row; a multiply by
+      // 2^(31 - 8 (c % 4) - t) moves it to bit 31 on the FMA pipe, leaving one AND-XOR
+      // (the integer pipe) and one add per element and block
+      uint32_t mq[4];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
-      const uint8_t* sbase = smem + L.s_off + sb * L.s_stride;
+      for (int q = 0; q < 4; ++q) mq[q] = 1u << (31 - 8 * q - t);
+      float acc[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
+      const uint8_t* sbase = smem + L.s_off + sb * L.s_stride + half * 2048 + tid * 16;
       for (int r = 0; r < rounds; ++r) {
-        if (!failed) check(mbar_wait(&ctl->pfull, static_cast<uint32_t>(prounds & 1), deadline, abort_flag));
+        const int g = prounds & 1;   // P rounds alternate between the two TMEM regions
+        if (!failed) check(mbar_wait(&ctl->pfull[g], static_cast<uint32_t>((prounds >> 1) & 1), deadline, abort_flag));
         if (!failed) {
           tc_fence_after();
           const int i1 = min(n, (r + 1) * kPRound);
           for (int i = r * kPRound; i < i1; ++i) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + kPcol + (i - r * kPRound) * 32, v);
-            const uint4 wa = *reinterpret_cast<const uint4*>(sbase + i * kTileBytes + tid * 16);
-            const uint4 wb = *reinterpret_cast<const uint4*>(sbase + i * kTileBytes + 2048 + tid * 16);
-            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + kPcol + 128u * g + (i - r * kPRound) * 32 + 16 * half, v);
+            const uint4 wq = *reinterpret_cast<const uint4*>(sbase + i * kTileBytes);
+            const uint32_t wd[4] = {wq.x, wq.y, wq.z, wq.w};
             tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              // column c of the K-tile is bit 8 (c % 4) + t of word c / 4
-              const uint32_t sgn = (wd[c >> 2] << (31 - (8 * (c & 3) + t))) & 0x80000000u;
-              acc[c] += __uint_as_float(v[c] ^ sgn);
+            for (int c = 0; c < 16; ++c) {
+              uint32_t x;
+              asm("mul.lo.u32 %0, %1, %2;" : "=r"(x) : "r"(wd[c >> 2]), "r"(mq[c & 3]));
+              acc[c] += __uint_as_float(v[c] ^ (x & 0x80000000u));
             }
           }
           tc_fence_before();
-          mbar_arrive(&ctl->pempty);
+          mbar_arrive(&ctl->pempty[g]);
         }
         ++prounds;
       }
       if (!failed && t == 7) mbar_arrive(&sgempty[sb]);
-      uint32_t packed[16];
+      uint32_t packed[8];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float s0 = __ldg(p.inv_s + kt * kKT + c), s1 = __ldg(p.inv_s + kt * kKT + c + 1);
-        packed[c / 2] = pack2<DT>(acc[c] * s0, acc[c + 1] * s1);
+      for (int c = 0; c < 16; c += 2) {
+        const int col = kt * kKT + 16 * half + c;
+        packed[c / 2] = pack2<DT>(acc[c] * __ldg(p.inv_s + col), acc[c + 1] * __ldg(p.inv_s + col + 1));
       }
       if (kt >= 2 && !failed) check(mbar_wait(&ctl->wempty[w], static_cast<uint32_t>(((kt >> 1) - 1) & 1), deadline, abort_flag));
       if (!failed) {
         uint8_t* wb = smem + L.w_off + w * kTileRows * kKT * 2;
 #pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int kc = 2 * half + k2;   // 8-column K chunk of the tile
           *reinterpret_cast<uint4*>(wb + kc * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
-              make_uint4(packed[4 * kc], packed[4 * kc + 1], packed[4 * kc + 2], packed[4 * kc + 3]);
+              make_uint4(packed[4 * k2], packed[4 * k2 + 1], packed[4 * k2 + 2], packed[4 * k2 + 3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&ctl->wfull[w]);
       }
     }
-    // epilogue: accumulator row `tid` holds NT token outputs
+    // epilogue: accumulator row `tid` holds NT token outputs; the two halves take
+    // alternate 32-column chunks
     if (!failed) check(mbar_wait(&ctl->accfull, 0, deadline, abort_flag));
     if (!failed) {
       tc_fence_after();
       DT* y = static_cast<DT*>(p.y);
       const size_t row = static_cast<size_t>(rt) * kTileRows + tid;
-      for (int ch = 0; ch < NT / 32; ++ch) {
+      for (int ch = half; ch < NT / 32; ch += 2) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + ch * 32, v);
         tc_wait_ld();
