@@ -208,6 +208,48 @@ bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_s
 /* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
 bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream);
 
+/* ----------------------------------------------------------- load planning ----- */
+
+/* Orders of the universal stack.  All blocks of all weights sit in one stack on the
+ * storage device and are loaded or offloaded in a presorted order as the memory
+ * budget changes (review page "BitStack: Fine-Grained Size Control...", Fig. 2
+ * caption; OpenReview discussion, reply A1.B); the review page's Fig. 6 compares an
+ * Average, a Greedy and a Random order. */
+typedef enum {
+  BS_ORDER_AVERAGE = 0, /* level-major: block 0 of every weight, then block 1, ...;
+                           weights in index order within a level */
+  BS_ORDER_GREEDY = 1,  /* repeatedly the weight whose next block has the highest
+                           score; equal scores: the lower weight index */
+  BS_ORDER_RANDOM = 2   /* step t: weight live[floor(draws[t] * |live|)] of the
+                           weights with blocks left, in index order */
+} bs_order_kind;
+
+/* Writes the global load order of sum(n_blocks) blocks: step t loads block
+ * out_block[t] of weight out_weight[t].  Within every weight the blocks come in
+ * their own order 0, 1, 2, ... (each residual block corrects what the earlier ones
+ * left; review page, Fig. 2), so only the interleaving of weights is chosen.
+ * n_blocks: n_weights counts >= 0.  scores (GREEDY only, else may be NULL): row w
+ *   holds weight w's per-block scores at scores[w * score_stride + i], i < n_blocks[w]
+ *   (score_stride >= max n_blocks).  A natural score is the drop of the weight's
+ *   scaled residual energy per byte, (|R_i|^2 - |R_{i+1}|^2) / block bytes.
+ * draws (RANDOM only, else may be NULL): sum(n_blocks) numbers in [0, 1), the
+ *   caller's random stream.
+ * out_weight, out_block: caller-owned host arrays of sum(n_blocks) ints.
+ * Host only; no device is touched.  BS_ERR_INVALID_ARG on null pointers the kind
+ * needs, negative counts, a stride below the largest count, a draw outside [0, 1),
+ * an unknown kind, or more than 2^30 blocks in total. */
+bs_status bs_plan_order(int n_weights, const int* n_blocks, const double* scores, int score_stride,
+                        bs_order_kind kind, const double* draws, int* out_weight, int* out_block);
+
+/* Loads the longest prefix of a load order that fits a byte budget: walks
+ * order_weight[0 .. n_steps) and counts a block of weight w (block_bytes[w] bytes)
+ * until the next one would take the total above budget_bytes, then stops.
+ * out_loaded: caller-owned array of n_weights ints, the blocks to keep loaded per
+ * weight (blocks 0 .. out_loaded[w]-1).  Host only.  BS_ERR_INVALID_ARG on null
+ * pointers, n_steps < 0, n_weights <= 0 or a weight index outside [0, n_weights). */
+bs_status bs_plan_budget(long long n_steps, const int* order_weight, int n_weights,
+                         const unsigned long long* block_bytes, unsigned long long budget_bytes, int* out_loaded);
+
 /* ------------------------------------------------------------------ errors ----- */
 
 /* Synchronises `stack`'s device, reads and clears the sticky device error word:

@@ -15,6 +15,10 @@ reading: matrix w has an importance weight a_w (seeded, from ``workloads``); blo
 The key grows with i for a fixed w, so the order keeps every weight's blocks in
 prefix order, as a per-weight stack requires.  Parity unpinned for the key itself;
 the prefix property and the budget fill are pinned by the tests.
+
+The importance-scored orders below (Greedy, Average, Random; Review, Fig. 6) are
+pinned by brute force over tiny stacks, a library sort, closed forms, hand-worked
+draws and residual energies recomputed from reconstructed weights.
 """
 from __future__ import annotations
 
@@ -53,3 +57,69 @@ def budget_fill(order, block_bytes_per_matrix, budget_mib: float) -> np.ndarray:
         used += int(sizes[w])
         n[w] += 1
     return n
+
+
+# ------------------------------------------------------------- importance scoring ----
+# The pages name three orders for the residual blocks of all weights (Review, Fig. 6
+# caption: Average, Greedy, Random) and a scoring step (README "Decomposition",
+# ``--score_importance``), but do not print the algorithm (Rebuttal A1.A refers to
+# Algorithm 1 of the paper).  Readings taken here:
+#   * score of block i of weight w: the drop it brings to the squared Frobenius norm
+#     of the weight's scaled residual, ||R_{i-1}||^2 - ||R_i||^2, per byte of the block
+#     record (the scaled domain carries the activation-aware weighting, Review Fig. 5);
+#   * Greedy: repeatedly load the next block (lowest unloaded index) of the weight
+#     whose next block scores highest (ties: lower weight index);
+#   * Average: every weight gets the same number of blocks, level by level (block 0
+#     of every weight in weight order, then block 1, ...);
+#   * Random: at each step one weight with blocks left is picked uniformly; the uniform
+#     draws are inputs (one per step), the pick is floor(u * count) among the weights
+#     with blocks left, in weight order.
+# Every order keeps each weight's blocks in prefix order, which a per-weight stack needs.
+
+
+def block_scores(res_norms, block_bytes: int) -> np.ndarray:
+    """Per-block score (float64): (||R_{i-1}||^2 - ||R_i||^2) / block_bytes from the
+    residual norms R_0, ..., R_n a decomposition records (``Decomposition.res_norms``)."""
+    r = np.asarray(res_norms, dtype=np.float64)
+    return (r[:-1] ** 2 - r[1:] ** 2) / float(block_bytes)
+
+
+def order_greedy(scores) -> list:
+    """[(weight, block)]: always the highest-scoring next block (ties: lower weight)."""
+    nxt = [0] * len(scores)
+    out = []
+    total = sum(len(s) for s in scores)
+    while len(out) < total:
+        best = None
+        for w, s in enumerate(scores):
+            if nxt[w] < len(s) and (best is None or float(s[nxt[w]]) > float(scores[best][nxt[best]])):
+                best = w
+        out.append((best, nxt[best]))
+        nxt[best] += 1
+    return out
+
+
+def order_average(counts) -> list:
+    """[(weight, block)] level by level: block i of every weight that has one, in
+    weight order, for i = 0, 1, ..."""
+    counts = [int(c) for c in counts]
+    out = []
+    for i in range(max(counts) if counts else 0):
+        for w, c in enumerate(counts):
+            if i < c:
+                out.append((w, i))
+    return out
+
+
+def order_random(counts, draws) -> list:
+    """[(weight, block)]: step t picks weight number floor(draws[t] * live) among the
+    ``live`` weights that still have blocks, in weight order."""
+    counts = [int(c) for c in counts]
+    nxt = [0] * len(counts)
+    out = []
+    for t in range(sum(counts)):
+        live = [w for w, c in enumerate(counts) if nxt[w] < c]
+        w = live[min(int(float(draws[t]) * len(live)), len(live) - 1)]
+        out.append((w, nxt[w]))
+        nxt[w] += 1
+    return out

@@ -31,11 +31,16 @@ BS_F16 = 0
 BS_BF16 = 1
 BS_F32 = 2
 
+BS_ORDER_AVERAGE = 0
+BS_ORDER_GREEDY = 1
+BS_ORDER_RANDOM = 2
+
 EXPORTS = (
     "bs_block_bytes", "bs_stack_device_bytes", "bs_workspace_bytes", "bs_pack_record",
     "bs_stack_create", "bs_stack_destroy", "bs_stack_num_blocks", "bs_append_block",
     "bs_drop_block", "bs_linear", "bs_reconstruct", "bs_unpack_signs",
     "bs_get_device_error", "bs_status_string", "bs_debug_set_wait", "bs_linear_no_alloc",
+    "bs_plan_order", "bs_plan_budget",
 )
 
 
@@ -67,6 +72,8 @@ def _load():
         "bs_status_string": (ctypes.c_char_p, [I]),
         "bs_debug_set_wait": (I, [P, LL, I]),
         "bs_linear_no_alloc": (I, [P, P, I, I, I, P, P]),
+        "bs_plan_order": (I, [I, P, P, I, I, P, P, P]),
+        "bs_plan_budget": (I, [LL, P, I, P, ctypes.c_ulonglong, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,3 +202,29 @@ def bs_get_device_error(handle: int) -> int:
 
 def bs_debug_set_wait(handle: int, timeout_ns: int, unreachable_flag: bool = False) -> None:
     _check(lib.bs_debug_set_wait(handle, int(timeout_ns), 1 if unreachable_flag else 0), "bs_debug_set_wait")
+
+
+def bs_plan_order(n_blocks, kind: int, scores=None, draws=None):
+    """Global load order of all blocks: two int32 arrays (weight, block) of
+    sum(n_blocks) entries.  ``scores`` is a (n_weights, >= max n_blocks) float64
+    array (GREEDY), ``draws`` sum(n_blocks) float64 numbers in [0, 1) (RANDOM)."""
+    counts = np.ascontiguousarray(n_blocks, dtype=np.int32)
+    total = int(counts.sum()) if counts.size else 0
+    out_w = np.zeros(max(total, 1), dtype=np.int32)
+    out_b = np.zeros(max(total, 1), dtype=np.int32)
+    sc = None if scores is None else np.ascontiguousarray(scores, dtype=np.float64)
+    dr = None if draws is None else np.ascontiguousarray(draws, dtype=np.float64)
+    stride = 0 if sc is None else (sc.shape[1] if sc.ndim == 2 else 0)
+    _check(lib.bs_plan_order(counts.size, _ptr(counts), _ptr(sc), stride, int(kind), _ptr(dr), _ptr(out_w),
+                             _ptr(out_b)), "bs_plan_order")
+    return out_w[:total], out_b[:total]
+
+
+def bs_plan_budget(order_weight, block_bytes, budget_bytes: int):
+    """Blocks per weight that the longest fitting prefix of ``order_weight`` loads."""
+    order = np.ascontiguousarray(order_weight, dtype=np.int32)
+    sizes = np.ascontiguousarray(block_bytes, dtype=np.uint64)
+    out = np.zeros(max(sizes.size, 1), dtype=np.int32)
+    _check(lib.bs_plan_budget(order.size, _ptr(order) if order.size else None, sizes.size, _ptr(sizes),
+                              int(budget_bytes), _ptr(out)), "bs_plan_budget")
+    return out[:sizes.size]

@@ -26,6 +26,7 @@ STREAMS = {
     "blocks": 5,     # synthetic residual blocks (signs and factors)
     "order": 6,      # per-matrix importance weights for the global block order
     "svd": 7,        # random test matrices for randomized SVD
+    "plan": 8,       # residual-norm decay per block for load-order planning
 }
 
 K_DEFAULT = 16
