@@ -64,6 +64,12 @@ constexpr int kNI = 3;                 // issuer warps (20 warps in all at batch
 constexpr int kBarZ = 4;               // named barriers: 4 = all warps but the copy warp, 5 = epilogue
 constexpr int kBarEpi = 5;
 constexpr float kQMax = 32512.0f;      // |q| <= 127 * 256: q = 256 hi + lo with hi, lo in int8
+// Rounding to an integer by addition: for |v| < 2^22, the float nearest to 1.5 * 2^23 + v
+// lies in [2^23, 2^24), where floats are the integers, so it is 1.5 * 2^23 + rint(v)
+// (ties to even: 1.5 * 2^23 is even), and its bit pattern is kRoundBits + rint(v).
+// kRoundBias adds 128 more, so the pattern is kRoundBits + q + 128.
+constexpr uint32_t kRoundBits = 0x4B400000u;   // bit pattern of 1.5 * 2^23
+constexpr float kRoundBias = 12583040.0f;      // 1.5 * 2^23 + 128
 
 template <int B>
 struct Cfg {
@@ -251,8 +257,8 @@ __device__ __forceinline__ Tv warp_reduce_scatter16(Tv (&v)[16], int lane, Op op
 struct MaxOp {
   __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
 };
-struct AddOp {
-  __device__ __forceinline__ int operator()(int a, int b) const { return a + b; }
+struct UAddOp {
+  __device__ __forceinline__ uint32_t operator()(uint32_t a, uint32_t b) const { return a + b; }
 };
 
 // The 16 fp16 entries of one V row (32 bytes) as fp32, from global memory (read-only
@@ -336,10 +342,14 @@ __device__ void set_quant(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* se
   const int lane = zt & 31;
 #pragma unroll
   for (int b = 0; b < B; ++b) {
-    const float* rlo = ctl->rlo[slot] + b * 16;   // shared-memory broadcast reads
-    int zs[16];
+    // 1 / step of the 16 columns in registers (the stores below go to shared memory too,
+    // so reads through a pointer would be repeated after every store)
+    float rl[16];
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) zs[jj] = 0;
+    for (int jj = 0; jj < 16; ++jj) rl[jj] = ctl->rlo[slot][b * 16 + jj];
+    uint32_t zs[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) zs[jj] = 0u;
     for (int c = zt; c < gcols; c += NT) {
       const float xv = x_scaled<kGlobal>(p, S, c, b);
       float v[16];
@@ -350,16 +360,19 @@ __device__ void set_quant(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* se
       uint8_t* base = set + cc * K::ZB + ((cl >> 5) * (NB / 8) * 2 + ((cl >> 4) & 1)) * 128 + (cl & 15);
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
-        // |Z| / sigma <= 32512 up to a rounding far below 1/2, so rint stays in range
-        const int q = __float2int_rn(__fmul_rn(xv, v[jj]) * rlo[jj]);
-        zs[jj] += q;
+        // q = rint(Z / sigma), |q| <= 32512 (the step makes |Z| / sigma <= 32512 up to a
+        // rounding far below 1/2): one fused multiply-add with kRoundBias leaves the bit
+        // pattern bq = kRoundBits + q + 128 (see kRoundBias), whose byte 1 is the hi
+        // plane (q + 128) >> 8 and whose byte 0, with bit 7 flipped, the lo plane q mod 256
+        const uint32_t bq = __float_as_uint(__fmaf_rn(__fmul_rn(xv, v[jj]), rl[jj], kRoundBias));
+        zs[jj] += bq;
         const int nh = b * 16 + jj, nl = NCOL + nh;
-        base[(nh >> 3) * 256 + (nh & 7) * 16] = static_cast<uint8_t>((q + 128) >> 8);   // hi
-        base[(nl >> 3) * 256 + (nl & 7) * 16] = static_cast<uint8_t>(q);                // lo = q - 256 hi, mod 256
+        base[(nh >> 3) * 256 + (nh & 7) * 16] = static_cast<uint8_t>(bq >> 8);      // hi
+        base[(nl >> 3) * 256 + (nl & 7) * 16] = static_cast<uint8_t>(bq ^ 0x80u);   // lo = q - 256 hi, mod 256
       }
     }
-    const int sum = warp_reduce_scatter16(zs, lane, AddOp());
-    if ((lane & 1) == 0) ctl->wpart[zt >> 5][b * 16 + scatter_index(lane)] = sum;
+    const uint32_t sum = warp_reduce_scatter16(zs, lane, UAddOp());
+    if ((lane & 1) == 0) ctl->wpart[zt >> 5][b * 16 + scatter_index(lane)] = static_cast<int>(sum);
   }
 }
 
@@ -385,9 +398,12 @@ __device__ void build_set(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* se
   fence_proxy_async_smem();   // the MMAs read the operand through the async proxy
   bar_named(bar, NT);
   if (zt < NCOL) {
-    int sum = 0;
-    for (int w = 0; w < nw; ++w) sum += ctl->wpart[w][zt];
-    ctl->csum[slot][zt] = sum;
+    // the partials hold sums of bq = q + kRoundBits + 128 (mod 2^32); the sum of q itself
+    // is below 2^31 in magnitude (at most 1024 columns of |q| <= 32512)
+    uint32_t sum = 0u;
+    for (int w = 0; w < nw; ++w) sum += static_cast<uint32_t>(ctl->wpart[w][zt]);
+    sum -= static_cast<uint32_t>(gcols) * (kRoundBits + 128u);
+    ctl->csum[slot][zt] = static_cast<int>(sum);
   }
   bar_named(bar, NT);
 }

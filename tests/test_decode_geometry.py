@@ -95,6 +95,9 @@ def test_shared_tensor_memory_and_threads_fit(b):
     # modulo 4 still cover the four tensor-memory lane quadrants once each
     wepi = 4 * K.T + K.NI
     assert sorted(w % 4 for w in range(wepi, wepi + 4)) == [0, 1, 2, 3]
+    # the row-tile reduction's scratch (4 tiles x slices x batch x 128 fp32, then the
+    # completed row-tile list) fits the drained sign stages
+    assert 4 * (K.THREADS // 128) * b * 128 * 4 + K.THREADS * 4 <= K.NS * K.STAGE
     # the activation sets sit at the start of shared memory: descriptor addresses fit
     # their 14-bit field (16-byte units)
     assert (2 * K.SET) >> 4 < (1 << 14)
