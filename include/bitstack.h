@@ -208,6 +208,41 @@ bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_s
 /* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
 bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream);
 
+/* ------------------------------------------- "w/o AVD" blocks (vanilla SVD) ----- */
+
+/* The ablation of the review page, Fig. 5 caption: every residual block is a plain
+ * rank-k' factor pair from the vanilla SVD of the residual (no sign matrix), with
+ * k' = k + m n / (16 (m + n)) so that a block takes the bytes of a BitStack block.
+ * Record: [U, m x k' fp16 row-major][V, d x k' fp16 row-major], 2 k' (m + d) bytes,
+ * sqrt(sigma) folded into both factors as for BitStack blocks.  Such a stack takes the
+ * same calls as a BitStack stack (append, drop, num_blocks, linear, reconstruct,
+ * get_device_error, destroy); bs_unpack_signs and bs_linear_no_alloc return
+ * BS_ERR_INVALID_ARG for it.  Shapes: any m, d in 1 .. 65536; k' a multiple of 8 in
+ * 8 .. 256 (whole 16-byte factor rows). */
+
+/* k' for an m x d weight and BitStack rank k: k + m d / (16 (m + d)) rounded down to a
+ * multiple of 8 (exact for 4096 x 4096, k = 16: 144).  0 on non-positive arguments. */
+int bs_plain_rank(int m, int d, int k);
+
+/* 2 k' (m + d); 0 for a shape outside the rules above. */
+size_t bs_plain_block_bytes(int m, int d, int k_prime);
+
+/* capacity * bs_plain_block_bytes rounded up to 256, plus 256 bytes for the stack's
+ * device error word; 0 on invalid arguments. */
+size_t bs_plain_stack_device_bytes(int m, int d, int k_prime, int capacity_blocks);
+
+/* Workspace bs_linear needs on a "w/o AVD" stack (0 for n_loaded == 0): n arrival
+ * counters, t = (x / s) V_i for up to 16 rows of x, and per-128-row slice parts of t,
+ * about 4 k' n (d / 128 + 1) min(batch, 16) bytes.  Zero it once before first use; every
+ * completed call leaves its counters at zero.  Any batch: x is taken in passes of 16
+ * rows, ordered on the stream, which reuse the workspace. */
+size_t bs_plain_workspace_bytes(int m, int d, int k_prime, int n_loaded, int batch);
+
+/* As bs_stack_create, for "w/o AVD" blocks of rank k_prime
+ * (dev_bytes >= bs_plain_stack_device_bytes). */
+bs_status bs_plain_stack_create(int m, int d, int k_prime, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                                const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out);
+
 /* ----------------------------------------------------------- load planning ----- */
 
 /* Orders of the universal stack.  All blocks of all weights sit in one stack on the

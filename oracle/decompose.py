@@ -138,7 +138,7 @@ class Decomposition:
 
     @property
     def n_blocks(self) -> int:
-        return len(self.neg)
+        return len(self.U)
 
 
 def avd_step(R: np.ndarray, k: int, gen: np.random.Generator | None = None,
@@ -206,6 +206,68 @@ def decompose(W: np.ndarray, s: np.ndarray, n_blocks: int, k: int,
         neg, U, V, R, sig = avd_step(R, k, gen, round_fp16, info=info)
         out.svd_info.append(info)
         out.neg.append(neg)
+        out.U.append(U)
+        out.V.append(V)
+        out.sigmas.append(sig)
+        out.res_norms.append(float(np.linalg.norm(R)))
+    return out
+
+
+# ------------------------------------------------------------ "w/o AVD" blocks ------
+def plain_rank(m: int, d: int, k: int) -> int:
+    """Rank k' of a vanilla-SVD block that takes the bytes of a BitStack block.
+
+    Follows: Review, Fig. 5 caption (the "w/o AVD" ablation sets k' = k + m n / (16
+    (m + n)) for an m x n weight so that a block keeps the size of the main
+    experiments' blocks).  Reading taken where the fraction is not whole: k' is
+    rounded down to a multiple of 8, so that the block never grows past the block it
+    stands in for and every factor row is a whole number of 16-byte units (the
+    library's layout).  For 4096 x 4096 and k = 16 the fraction is whole: k' = 144,
+    and 2 k' (m + d) = m d / 8 + 2 k (m + d) exactly.
+    """
+    kp = k + (m * d) // (16 * (m + d))
+    return kp - kp % 8
+
+
+def plain_step(R: np.ndarray, kp: int, gen: np.random.Generator | None = None,
+               round_fp16: bool = True, info: dict | None = None):
+    """One vanilla-SVD residual block: the rank-k' truncated SVD of the residual R
+    itself (signed, no sign matrix), sqrt(sigma) folded into both fp16 factors as in
+    avd_step.
+
+    Follows: Review, Fig. 5 caption ("w/o AVD": vanilla SVD, Eq. 5, replaces the
+    absolute value decomposition; the iteration over residuals is unchanged).
+    Returns (U, V, R_next, sigma) with R_next = R - U V^T from the stored factors.
+    """
+    Ut, sig, Vt = truncated_svd(R, kp, gen, info=info)
+    root = np.sqrt(sig)
+    U = Ut * root[None, :]
+    V = Vt.T * root[None, :]
+    if round_fp16:
+        U16, V16 = U.astype(np.float16), V.astype(np.float16)
+        Ue, Ve = U16.astype(np.float64), V16.astype(np.float64)
+    else:
+        U16, V16 = U, V
+        Ue, Ve = U, V
+    return U16, V16, R - Ue @ Ve.T, sig
+
+
+def decompose_plain(W: np.ndarray, s: np.ndarray, n_blocks: int, kp: int,
+                    gen: np.random.Generator | None = None, round_fp16: bool = True) -> Decomposition:
+    """The "w/o AVD" decomposition: as ``decompose`` (activation-aware scaling, then one
+    block per iteration on the previous residual), with plain_step in place of
+    avd_step.  The result has no sign matrices (``neg`` stays empty)."""
+    W = np.asarray(W, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    out = Decomposition()
+    out.s = s.copy()
+    out.inv_s = (1.0 / s).astype(np.float32)
+    R = W * s[None, :]
+    out.res_norms.append(float(np.linalg.norm(R)))
+    for _ in range(n_blocks):
+        info: dict = {}
+        U, V, R, sig = plain_step(R, kp, gen, round_fp16, info=info)
+        out.svd_info.append(info)
         out.U.append(U)
         out.V.append(V)
         out.sigmas.append(sig)

@@ -111,3 +111,52 @@ def linear_rows(x: np.ndarray, negs, Us, Vs, inv_s, n: int, rows: np.ndarray) ->
             w += _signs(negs[i][r]) * p
         out[:, idx] = x @ (w * inv_s)
     return out
+
+
+# ------------------------------------------------------------ "w/o AVD" blocks ------
+def reconstruct_plain(Us, Vs, inv_s, n: int, m: int) -> np.ndarray:
+    """W_hat_n = (sum_{i < n} U_i V_i^T) diag(1/s) for vanilla-SVD blocks (float64).
+
+    Follows: Review, Fig. 5 caption ("w/o AVD" blocks are plain low-rank factors, the
+    scaling undone per input channel as for BitStack blocks).
+    """
+    inv_s = np.asarray(inv_s, dtype=np.float64)
+    W = np.zeros((m, inv_s.shape[0]), dtype=np.float64)
+    for i in range(n):
+        W += np.asarray(Us[i], dtype=np.float64) @ np.asarray(Vs[i], dtype=np.float64).T
+    return W * inv_s[None, :]
+
+
+def linear_plain_explicit(x: np.ndarray, Us, Vs, inv_s, n: int, m: int) -> np.ndarray:
+    """y = x W_hat_n^T (float64 b x m) with W_hat_n from reconstruct_plain."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    return x @ reconstruct_plain(Us, Vs, inv_s, n, m).T
+
+
+def linear_plain_factored(x: np.ndarray, Us, Vs, inv_s, n: int, m: int) -> np.ndarray:
+    """y = sum_i ((x * 1/s) V_i) U_i^T (float64 b x m): the same value by
+    associativity, never forming the weight."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    y = np.zeros((x.shape[0], m), dtype=np.float64)
+    xs = x * np.asarray(inv_s, dtype=np.float64)[None, :]
+    for i in range(n):
+        t = xs @ np.asarray(Vs[i], dtype=np.float64)
+        y += t @ np.asarray(Us[i], dtype=np.float64).T
+    return y
+
+
+def linear_plain_bruteforce(x, Us, Vs, inv_s, n: int, m: int) -> np.ndarray:
+    """Pure-Python loops over (b, r, c, i, j); tiny shapes only."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    bsz, d = x.shape
+    y = np.zeros((bsz, m), dtype=np.float64)
+    for b in range(bsz):
+        for r in range(m):
+            acc = 0.0
+            for c in range(d):
+                xc = float(x[b, c]) * float(inv_s[c])
+                for i in range(n):
+                    for j in range(Us[i].shape[1]):
+                        acc += xc * float(Us[i][r, j]) * float(Vs[i][c, j])
+            y[b, r] = acc
+    return y

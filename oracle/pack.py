@@ -130,3 +130,17 @@ def parse_record(rec: np.ndarray, m: int, d: int, k: int):
     U = rec[nsb:nsb + 2 * m * k].view(np.float16).reshape(m, k)
     V = rec[nsb + 2 * m * k:nsb + 2 * k * (m + d)].view(np.float16).reshape(d, k)
     return unpack_device(words, m, d), U, V
+
+
+def plain_block_bytes(m: int, d: int, kp: int) -> int:
+    """Bytes of one vanilla-SVD ("w/o AVD") block record: 2 k' (m + d) (fp16 U, V)."""
+    return 2 * kp * (m + d)
+
+
+def make_plain_record(U: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """The "w/o AVD" record bytes (uint8): U (m x k' fp16 row-major), then V (d x k')."""
+    U = np.ascontiguousarray(U, dtype=np.float16)
+    V = np.ascontiguousarray(V, dtype=np.float16)
+    if U.shape[1] != V.shape[1]:
+        raise ValueError("U and V ranks differ")
+    return np.concatenate([U.view(np.uint8).reshape(-1), V.view(np.uint8).reshape(-1)])

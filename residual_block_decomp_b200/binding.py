@@ -40,7 +40,8 @@ EXPORTS = (
     "bs_stack_create", "bs_stack_destroy", "bs_stack_num_blocks", "bs_append_block",
     "bs_drop_block", "bs_linear", "bs_reconstruct", "bs_unpack_signs",
     "bs_get_device_error", "bs_status_string", "bs_debug_set_wait", "bs_linear_no_alloc",
-    "bs_plan_order", "bs_plan_budget",
+    "bs_plan_order", "bs_plan_budget", "bs_plain_rank", "bs_plain_block_bytes", "bs_plain_stack_device_bytes",
+    "bs_plain_workspace_bytes", "bs_plain_stack_create",
 )
 
 
@@ -74,6 +75,11 @@ def _load():
         "bs_linear_no_alloc": (I, [P, P, I, I, I, P, P]),
         "bs_plan_order": (I, [I, P, P, I, I, P, P, P]),
         "bs_plan_budget": (I, [LL, P, I, P, ctypes.c_ulonglong, P]),
+        "bs_plain_rank": (I, [I, I, I]),
+        "bs_plain_block_bytes": (Z, [I, I, I]),
+        "bs_plain_stack_device_bytes": (Z, [I, I, I, I]),
+        "bs_plain_workspace_bytes": (Z, [I, I, I, I, I]),
+        "bs_plain_stack_create": (I, [I, I, I, I, P, Z, P, P, ctypes.POINTER(P)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -151,6 +157,31 @@ def bs_stack_create(m: int, d: int, k: int, capacity: int, dev_blocks, inv_scale
     st = lib.bs_stack_create(m, d, k, capacity, _ptr(dev_blocks), dev_blocks.numel() * dev_blocks.element_size(),
                              _ptr(inv_scale), _stream(stream), ctypes.byref(h))
     _check(st, "bs_stack_create")
+    return h.value
+
+
+def bs_plain_rank(m: int, d: int, k: int) -> int:
+    return int(lib.bs_plain_rank(m, d, k))
+
+
+def bs_plain_block_bytes(m: int, d: int, k_prime: int) -> int:
+    return int(lib.bs_plain_block_bytes(m, d, k_prime))
+
+
+def bs_plain_stack_device_bytes(m: int, d: int, k_prime: int, capacity: int) -> int:
+    return int(lib.bs_plain_stack_device_bytes(m, d, k_prime, capacity))
+
+
+def bs_plain_workspace_bytes(m: int, d: int, k_prime: int, n_loaded: int, batch: int) -> int:
+    return int(lib.bs_plain_workspace_bytes(m, d, k_prime, n_loaded, batch))
+
+
+def bs_plain_stack_create(m: int, d: int, k_prime: int, capacity: int, dev_blocks, inv_scale, stream=None) -> int:
+    h = ctypes.c_void_p()
+    st = lib.bs_plain_stack_create(m, d, k_prime, capacity, _ptr(dev_blocks),
+                                   dev_blocks.numel() * dev_blocks.element_size(), _ptr(inv_scale), _stream(stream),
+                                   ctypes.byref(h))
+    _check(st, "bs_plain_stack_create")
     return h.value
 
 

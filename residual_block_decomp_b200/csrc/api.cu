@@ -17,6 +17,11 @@ bool gpu_shape_ok(int m, int d, int k) {
          d % kTileCols == 0;
 }
 
+// "w/o AVD" stacks: any m, d; k' a multiple of 8 (whole 16-byte factor rows) up to 256.
+bool plain_shape_ok(int m, int d, int kp) {
+  return m >= 1 && d >= 1 && m <= 65536 && d <= 65536 && kp >= 8 && kp <= kPlainMaxRank && kp % 8 == 0;
+}
+
 // After the block area: the stack's device error word (256 bytes reserved).
 size_t meta_bytes(int /*capacity*/) { return 256; }
 
@@ -120,14 +125,20 @@ bs_status bs_pack_record(int m, int d, int k, const uint8_t* neg_bits, const uin
   return BS_OK;
 }
 
-bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
-                          const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out) {
+}  // extern "C"
+
+namespace {
+
+bs_status create_stack(int plain, int m, int d, int k, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                       const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out) {
   if (out == nullptr || dev_blocks == nullptr || dev_inv_scale == nullptr || capacity_blocks <= 0)
     return BS_ERR_INVALID_ARG;
   *out = nullptr;
-  if (!gpu_shape_ok(m, d, k)) return BS_ERR_UNSUPPORTED_SHAPE;
+  if (plain ? !plain_shape_ok(m, d, k) : !gpu_shape_ok(m, d, k)) return BS_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(dev_blocks, 256) || !aligned(dev_inv_scale, 16)) return BS_ERR_ALIGNMENT;
-  if (dev_bytes < bs_stack_device_bytes(m, d, k, capacity_blocks)) return BS_ERR_CAPACITY;
+  const size_t need = plain ? bs_plain_stack_device_bytes(m, d, k, capacity_blocks)
+                            : bs_stack_device_bytes(m, d, k, capacity_blocks);
+  if (dev_bytes < need) return BS_ERR_CAPACITY;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BS_ERR_NO_DEVICE;
   int major = 0, minor = 0, sms = 0;
@@ -138,13 +149,14 @@ bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_bl
   if (major != 10 || minor != 0) return BS_ERR_NO_DEVICE;
   bs_stack_s* s = new (std::nothrow) bs_stack_s();
   if (s == nullptr) return BS_ERR_INVALID_ARG;
+  s->plain = plain;
   s->m = m;
   s->d = d;
   s->k = k;
   s->capacity = capacity_blocks;
   s->n_blocks = 0;
   s->blocks = static_cast<uint8_t*>(dev_blocks);
-  s->block_bytes = bs_block_bytes(m, d, k);
+  s->block_bytes = plain ? bs_plain_block_bytes(m, d, k) : bs_block_bytes(m, d, k);
   s->dev_bytes = dev_bytes;
   s->inv_s = dev_inv_scale;
   s->err = reinterpret_cast<uint32_t*>(s->blocks + align_up(static_cast<size_t>(capacity_blocks) * s->block_bytes, 256));
@@ -152,7 +164,7 @@ bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_bl
   s->sm_count = sms;
   s->timeout_ns = 500000000ull;
   s->inject_unreachable = 0;
-  s->tmaps_ready = build_factor_maps(s) ? 1 : 0;
+  s->tmaps_ready = plain ? 0 : (build_factor_maps(s) ? 1 : 0);
   const cudaError_t e = cudaMemsetAsync(s->err, 0, meta_bytes(capacity_blocks), stream);
   if (e != cudaSuccess) {
     delete s;
@@ -160,6 +172,73 @@ bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_bl
   }
   *out = s;
   return BS_OK;
+}
+
+// bs_linear for a "w/o AVD" stack: x in passes of up to kPlainRowsPerPass rows.
+bs_status plain_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded, void* y,
+                       void* workspace, size_t workspace_bytes, bs_stream_t stream) {
+  const PlainWs L = plain_ws_layout(stack->d, stack->k, n_loaded, batch);
+  if (workspace == nullptr || workspace_bytes < L.total) return BS_ERR_CAPACITY;
+  if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  PlainParams p{};
+  p.blocks = stack->blocks;
+  p.block_bytes = stack->block_bytes;
+  p.v_off = static_cast<unsigned long long>(stack->m) * stack->k * 2;
+  p.x = x;
+  p.y = y;
+  p.inv_s = stack->inv_s;
+  p.part = reinterpret_cast<float*>(ws + L.part);
+  p.t = reinterpret_cast<float*>(ws + L.t);
+  p.cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  p.m = stack->m;
+  p.d = stack->d;
+  p.n = n_loaded;
+  p.kp = stack->k;
+  p.x_bf16 = dt == BS_BF16 ? 1 : 0;
+  for (int row0 = 0; row0 < batch; row0 += kPlainRowsPerPass) {
+    p.row0 = row0;
+    p.nb = batch - row0 < kPlainRowsPerPass ? batch - row0 : kPlainRowsPerPass;
+    const cudaError_t e = launch_plain(p, stream);
+    if (e != cudaSuccess) return BS_ERR_CUDA;
+  }
+  return BS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bs_status bs_stack_create(int m, int d, int k, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                          const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out) {
+  return create_stack(0, m, d, k, capacity_blocks, dev_blocks, dev_bytes, dev_inv_scale, stream, out);
+}
+
+int bs_plain_rank(int m, int d, int k) {
+  if (m <= 0 || d <= 0 || k <= 0) return 0;
+  const long long kp = k + (static_cast<long long>(m) * d) / (16ll * (static_cast<long long>(m) + d));
+  return static_cast<int>(kp - kp % 8);
+}
+
+size_t bs_plain_block_bytes(int m, int d, int k_prime) {
+  if (!plain_shape_ok(m, d, k_prime)) return 0;
+  return static_cast<size_t>(2) * k_prime * (static_cast<size_t>(m) + d);
+}
+
+size_t bs_plain_stack_device_bytes(int m, int d, int k_prime, int capacity_blocks) {
+  if (!plain_shape_ok(m, d, k_prime) || capacity_blocks <= 0) return 0;
+  return align_up(static_cast<size_t>(capacity_blocks) * bs_plain_block_bytes(m, d, k_prime), 256) +
+         meta_bytes(capacity_blocks);
+}
+
+size_t bs_plain_workspace_bytes(int m, int d, int k_prime, int n_loaded, int batch) {
+  if (!plain_shape_ok(m, d, k_prime) || n_loaded <= 0 || batch <= 0) return 0;
+  return plain_ws_layout(d, k_prime, n_loaded, batch).total;
+}
+
+bs_status bs_plain_stack_create(int m, int d, int k_prime, int capacity_blocks, void* dev_blocks, size_t dev_bytes,
+                                const float* dev_inv_scale, bs_stream_t stream, bs_stack_t* out) {
+  return create_stack(1, m, d, k_prime, capacity_blocks, dev_blocks, dev_bytes, dev_inv_scale, stream, out);
 }
 
 bs_status bs_stack_destroy(bs_stack_t stack) {
@@ -199,6 +278,7 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   if (!aligned(x, 16) || !aligned(y, 16)) return BS_ERR_ALIGNMENT;
   const int m = stack->m, d = stack->d;
   if (n_loaded == 0) return cuda_status(cudaMemsetAsync(y, 0, static_cast<size_t>(batch) * m * 2, stream));
+  if (stack->plain) return plain_linear(stack, x, batch, dt, n_loaded, y, workspace, workspace_bytes, stream);
 
   if (batch <= kDecodeMaxBatch) {
     if (n_loaded > kDecodeMaxBlocks) return BS_ERR_RANGE;
@@ -275,12 +355,16 @@ bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_s
   if (!aligned(W_out, 16)) return BS_ERR_ALIGNMENT;
   const size_t elems = static_cast<size_t>(stack->m) * stack->d;
   if (n == 0) return cuda_status(cudaMemsetAsync(W_out, 0, elems * (dt == BS_F32 ? 4 : 2), stream));
+  if (stack->plain)
+    return cuda_status(launch_plain_reconstruct(stack->blocks, stack->block_bytes,
+                                                static_cast<size_t>(stack->m) * stack->k * 2, stack->inv_s, stack->m,
+                                                stack->d, stack->k, n, W_out, dt, stream));
   return cuda_status(
       launch_reconstruct(stack->blocks, stack->block_bytes, stack->inv_s, stack->m, stack->d, n, W_out, dt, stream));
 }
 
 bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream) {
-  if (stack == nullptr || out == nullptr) return BS_ERR_INVALID_ARG;
+  if (stack == nullptr || out == nullptr || stack->plain) return BS_ERR_INVALID_ARG;
   if (block < 0 || block >= stack->n_blocks) return BS_ERR_RANGE;
   return cuda_status(launch_unpack(stack->blocks + static_cast<size_t>(block) * stack->block_bytes, stack->m,
                                    stack->d, out, stream));
@@ -300,7 +384,9 @@ const char* bs_status_string(bs_status status) {
   switch (status) {
     case BS_OK: return "ok";
     case BS_ERR_INVALID_ARG: return "invalid argument";
-    case BS_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need m % 128 == 0, d % 256 == 0, k == 16)";
+    case BS_ERR_UNSUPPORTED_SHAPE:
+      return "unsupported shape (BitStack blocks: m % 128 == 0, d % 256 == 0, k == 16; plain blocks: k' a multiple "
+             "of 8 up to 256)";
     case BS_ERR_ALIGNMENT: return "misaligned pointer";
     case BS_ERR_CAPACITY: return "capacity or buffer size exceeded";
     case BS_ERR_RANGE: return "block count or index out of range";

@@ -79,6 +79,32 @@ struct PrefillParams {
   unsigned long long timeout_ns;
 };
 
+// "w/o AVD" stacks: blocks that are plain rank-k' factor pairs, record = [U m x k' fp16
+// row-major][V d x k' fp16 row-major].  k' is a multiple of 8 (whole 16-byte rows), at
+// most kPlainMaxRank; bs_linear takes x in passes of up to kPlainRowsPerPass rows.
+constexpr int kPlainMaxRank = 256;
+constexpr int kPlainRowsPerPass = 16;
+struct PlainWs {
+  size_t cnt, t, part, total;   // [n] counters, [n][rows][k'] t, [slices][n][rows][k'] slice parts
+};
+PlainWs plain_ws_layout(int d, int kp, int n, int batch);
+struct PlainParams {
+  const uint8_t* blocks;
+  unsigned long long block_bytes;
+  unsigned long long v_off;    // V inside a record: m * k' * 2
+  const void* x;               // batch x d; this pass reads rows row0 .. row0 + nb - 1
+  void* y;                     // batch x m, same dtype
+  const float* inv_s;
+  float* part;
+  float* t;
+  uint32_t* cnt;
+  int m, d, n, kp, row0, nb, x_bf16;
+};
+cudaError_t launch_plain(const PlainParams& p, cudaStream_t stream);
+cudaError_t launch_plain_reconstruct(const uint8_t* blocks, unsigned long long block_bytes, size_t v_off,
+                                     const float* inv_s, int m, int d, int kp, int n, void* out, int dtype,
+                                     cudaStream_t stream);
+
 // Launchers (decode.cu, prefill.cu, aux_kernels.cu).  They return cudaSuccess or the
 // launch error.
 cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream);
@@ -101,6 +127,7 @@ cudaError_t launch_unpack(const uint8_t* record, int m, int d, int8_t* out, cuda
 
 // The handle.  Host memory only.
 struct bs_stack_s {
+  int plain;                   // 1: "w/o AVD" blocks (k holds k'), 0: BitStack blocks
   int m, d, k, capacity, n_blocks;
   uint8_t* blocks;
   size_t block_bytes, dev_bytes;

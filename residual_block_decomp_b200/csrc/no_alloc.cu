@@ -67,7 +67,7 @@ void note_device_error(int device) {
 extern "C" bs_status bs_linear_no_alloc(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int n_loaded,
                                         void* y, bs_stream_t stream) {
   if (stack == nullptr || x == nullptr || y == nullptr || batch <= 0) return BS_ERR_INVALID_ARG;
-  if (batch > bs::kDecodeMaxBatch) return BS_ERR_INVALID_ARG;
+  if (batch > bs::kDecodeMaxBatch || stack->plain) return BS_ERR_INVALID_ARG;
   if (n_loaded < 0 || n_loaded > stack->n_blocks) return BS_ERR_RANGE;
   const size_t need = bs::decode_ws_layout(stack->m, stack->d, n_loaded > 0 ? n_loaded : 1, batch).total;
   if (need > kStaticScratchBytes) return BS_ERR_CAPACITY;

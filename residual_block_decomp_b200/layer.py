@@ -19,23 +19,26 @@ class BitStackLinear:
 
     Parameters
     ----------
-    m, d : out_features, in_features (m % 128 == 0, d % 256 == 0)
+    m, d : out_features, in_features (m % 128 == 0, d % 256 == 0 for BitStack blocks)
     capacity : the most blocks the device area holds
     inv_scale : length-d float32 1/s of the activation-aware scaling
-    k : singular vectors per block (16 on the GPU path)
+    k : singular vectors per block (16 on the GPU path; k' for plain blocks)
+    plain : the blocks are "w/o AVD" rank-k' factor pairs (vanilla SVD, no signs)
     """
 
     def __init__(self, m: int, d: int, capacity: int, inv_scale, k: int = 16, device: str | int = "cuda",
-                 stream=None):
+                 stream=None, plain: bool = False):
         self.m, self.d, self.k, self.capacity = int(m), int(d), int(k), int(capacity)
+        self.plain = bool(plain)
         self.device = torch.device(device)
-        nbytes = B.bs_stack_device_bytes(m, d, k, capacity)
+        nbytes = (B.bs_plain_stack_device_bytes if plain else B.bs_stack_device_bytes)(m, d, k, capacity)
         if nbytes == 0:
             raise B.BsError(B.BS_ERR_UNSUPPORTED_SHAPE, "BitStackLinear")
         self.dev_blocks = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.inv_scale = torch.as_tensor(np.asarray(inv_scale, dtype=np.float32)).to(self.device).contiguous()
-        self.block_bytes = B.bs_block_bytes(m, d, k)
-        self.handle = B.bs_stack_create(m, d, k, capacity, self.dev_blocks, self.inv_scale, stream)
+        self.block_bytes = (B.bs_plain_block_bytes if plain else B.bs_block_bytes)(m, d, k)
+        create = B.bs_plain_stack_create if plain else B.bs_stack_create
+        self.handle = create(m, d, k, capacity, self.dev_blocks, self.inv_scale, stream)
         self.host_records: list[torch.Tensor] = []   # the storage copy of every block, pinned
         self._inflight: list[torch.Tensor] = []
         self._ws: torch.Tensor | None = None
@@ -75,7 +78,8 @@ class BitStackLinear:
             self.drop()
 
     def workspace(self, n_loaded: int, batch: int) -> torch.Tensor | None:
-        need = B.bs_workspace_bytes(self.m, self.d, self.k, n_loaded, batch)
+        need = (B.bs_plain_workspace_bytes if self.plain else B.bs_workspace_bytes)(self.m, self.d, self.k,
+                                                                                     n_loaded, batch)
         if need == 0:
             return None
         if self._ws is None or self._ws.numel() < need:
