@@ -204,56 +204,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_g = make_idesc(1u, is_bf16, is_bf16, 128u, static_cast<uint32_t>(NT));
       bool ok = mbar_wait(&ctl->ubar, 0, deadline, abort_flag);
       bool issued_any = false;
-      // Two streams from one thread: P rounds (rank-16 products of kPRound blocks into the
-      // two TMEM regions, as far ahead as a free region and a loaded V stage allow) and
-      // the GEMM of each K-tile once its W_hat tile is in shared memory.  Non-blocking
-      // barrier tests decide which goes next, so the products of the next rounds are
-      // computed while the rebuild warps read the current ones.
-      const int PR = KT * rounds;
-      int pr = 0, kg = 0;
+      // P round pr = (K-tile, round) into TMEM region pr & 1: rank-16 products of up to
+      // kPRound blocks, once the K-tile's V rows have landed and the rebuild warps have
+      // read the region's previous round.
       const uint32_t uaddr = smem_u32(smem + L.u_off);
-      for (uint32_t spins = 0; ok && kg < KT;) {
-        bool progressed = false;
-        if (pr < PR) {
-          const int ktp = pr / rounds, r = pr - ktp * rounds, s = ktp % XS, g = pr & 1;
-          if (mbar_test(&xfull[s], static_cast<uint32_t>((ktp / XS) & 1)) &&
-              (pr < 2 || mbar_test(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1)))) {
-            tc_fence_after();
-            const uint32_t vaddr = smem_u32(smem + L.v_off + s * L.v_stride);
-            const int i1 = min(n, (r + 1) * kPRound);
-            for (int i = r * kPRound; i < i1; ++i) {
-              const uint64_t adesc = smem_desc_noswizzle(uaddr + i * 4096, 2048, 128);
-              const uint64_t bdesc = smem_desc_noswizzle(vaddr + i * 1024, 512, 128);
-              mma_f16_ss(tmem + kPcol + 128u * g + (i - r * kPRound) * 32, adesc, bdesc, idesc_p, 0u);
-            }
-            issued_any = true;
-            tc_commit(&ctl->pfull[g]);
-            ++pr;
-            progressed = true;
-          }
+      auto issue_p = [&](int pr) -> bool {
+        const int ktp = pr / rounds, r = pr - ktp * rounds, s = ktp % XS, g = pr & 1;
+        if (!mbar_wait(&xfull[s], static_cast<uint32_t>((ktp / XS) & 1), deadline, abort_flag)) return false;
+        if (pr >= 2 && !mbar_wait(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1), deadline, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(smem + L.v_off + s * L.v_stride);
+        const int i1 = min(n, (r + 1) * kPRound);
+        for (int i = r * kPRound; i < i1; ++i) {
+          const uint64_t adesc = smem_desc_noswizzle(uaddr + i * 4096, 2048, 128);
+          const uint64_t bdesc = smem_desc_noswizzle(vaddr + i * 1024, 512, 128);
+          mma_f16_ss(tmem + kPcol + 128u * g + (i - r * kPRound) * 32, adesc, bdesc, idesc_p, 0u);
         }
+        issued_any = true;
+        tc_commit(&ctl->pfull[g]);
+        return true;
+      };
+      // One thread, a fixed order whose every wait is for an event the other warps produce
+      // without waiting on a later step of this thread: the P rounds of K-tile kg + 1
+      // (their regions free up as the rebuild warps finish the rounds of kg), then the
+      // GEMM of K-tile kg once its W_hat tile is in shared memory.  Blocking waits keep
+      // this thread off the issue slots the rebuild warps need.
+      const int PR = KT * rounds;
+      int pr = 0;
+      for (; pr < rounds && ok; ++pr) ok = issue_p(pr);
+      for (int kg = 0; kg < KT && ok; ++kg) {
+        for (; pr < min(PR, (kg + 2) * rounds) && ok; ++pr) ok = issue_p(pr);
         const int w = kg & 1;
-        if (kg * rounds < pr && mbar_test(&ctl->wfull[w], static_cast<uint32_t>((kg >> 1) & 1))) {
-          tc_fence_after();
-          const int s = kg % XS;
-          const uint32_t waddr = smem_u32(smem + L.w_off + w * kTileRows * kKT * 2);
-          const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
-          for (int kk = 0; kk < 2; ++kk) {
-            const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
-            const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
-            mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&ctl->wempty[w]);
-          tc_commit(&xempty[s]);   // the stage's V rows (read by this K-tile's P rounds) and x tile
-          ++kg;
-          progressed = true;
+        if (ok) ok = mbar_wait(&ctl->wfull[w], static_cast<uint32_t>((kg >> 1) & 1), deadline, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const int s = kg % XS;
+        const uint32_t waddr = smem_u32(smem + L.w_off + w * kTileRows * kKT * 2);
+        const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
+          const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
+          mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
         }
-        if (progressed) {
-          spins = 0;
-        } else if ((++spins & 63u) == 0u) {
-          if (*abort_flag || globaltimer_ns() > deadline) ok = false;
-          __nanosleep(20);
-        }
+        tc_commit(&ctl->wempty[w]);
+        tc_commit(&xempty[s]);   // the stage's V rows (read by this K-tile's P rounds) and x tile
       }
       if (ok) {
         tc_commit(&ctl->accfull);
@@ -286,6 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mq[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) mq[q] = 1u << (31 - 8 * q - t);
+      // 1/s of this thread's 16 columns, loaded before the waits so that their latency
+      // hides behind the rounds
+      float isv[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) isv[c] = __ldg(p.inv_s + kt * kKT + 16 * half + c);
       float acc[16];
 #pragma unroll
       for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
@@ -317,10 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!failed && t == 7) mbar_arrive(&sgempty[sb]);
       uint32_t packed[8];
 #pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const int col = kt * kKT + 16 * half + c;
-        packed[c / 2] = pack2<DT>(acc[c] * __ldg(p.inv_s + col), acc[c + 1] * __ldg(p.inv_s + col + 1));
-      }
+      for (int c = 0; c < 16; c += 2) packed[c / 2] = pack2<DT>(acc[c] * isv[c], acc[c + 1] * isv[c + 1]);
       if (kt >= 2 && !failed) check(mbar_wait(&ctl->wempty[w], static_cast<uint32_t>(((kt >> 1) - 1) & 1), deadline, abort_flag));
       if (!failed) {
         uint8_t* wb = smem + L.w_off + w * kTileRows * kKT * 2;
