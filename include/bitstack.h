@@ -208,6 +208,34 @@ bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_s
 /* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
 bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream);
 
+/* ------------------------------------------------- grouped decode (one launch) --- */
+
+/* A decode token through many linears in one launch.  The pages' use case is a whole
+ * model whose weights each hold a different number of loaded blocks, set by a memory
+ * budget over the universal block stack (review page "BitStack: Fine-Grained Size
+ * Control...", Fig. 2 caption; OpenReview discussion, reply A1.B); one launch over a
+ * table of all its linears replaces one launch per linear.  The work of all linears is
+ * split across the SMs as one list, so small and large linears share the machine.
+ *
+ * Workspace for bs_linear_group: the row-tile counters of all linears first (their
+ * places depend only on the shapes, so a workspace stays valid as n_loaded changes
+ * between tokens), then each linear's partials (about m d n batch / 256 bytes at batch
+ * 1).  Zero it once before first use; completed calls leave the counters at zero.
+ * 0 on invalid arguments (n_linears outside 1 .. 256, batch outside 1 .. 4, a null or
+ * "w/o AVD" stack, a negative count). */
+size_t bs_group_workspace_bytes(int n_linears, const bs_stack_t* stacks, const int* n_loaded, int batch);
+
+/* y[l] = x[l] W_hat_{n_loaded[l]}(stacks[l])^T for l < n_linears (<= 256), every x[l]
+ * batch x d_l and y[l] batch x m_l in one dtype, batch 1 .. 4, in one decode launch
+ * (plus one cudaMemsetAsync per linear with n_loaded[l] == 0).  Host arrays of
+ * n_linears entries, caller-owned.  All stacks must be BitStack stacks on the current
+ * device.  Results are bit-identical to one bs_linear call per linear.  A bounded wait
+ * that runs out is reported on stacks[0] (bs_get_device_error); zero the workspace
+ * again after that.  Errors as bs_linear, checked for every linear before any launch. */
+bs_status bs_linear_group(int n_linears, const bs_stack_t* stacks, const void* const* x, void* const* y,
+                          const int* n_loaded, int batch, bs_dtype dt, void* workspace, size_t workspace_bytes,
+                          bs_stream_t stream);
+
 /* ------------------------------------------- "w/o AVD" blocks (vanilla SVD) ----- */
 
 /* The ablation of the review page, Fig. 5 caption: every residual block is a plain

@@ -41,7 +41,7 @@ EXPORTS = (
     "bs_drop_block", "bs_linear", "bs_reconstruct", "bs_unpack_signs",
     "bs_get_device_error", "bs_status_string", "bs_debug_set_wait", "bs_linear_no_alloc",
     "bs_plan_order", "bs_plan_budget", "bs_plain_rank", "bs_plain_block_bytes", "bs_plain_stack_device_bytes",
-    "bs_plain_workspace_bytes", "bs_plain_stack_create",
+    "bs_plain_workspace_bytes", "bs_plain_stack_create", "bs_group_workspace_bytes", "bs_linear_group",
 )
 
 
@@ -80,6 +80,8 @@ def _load():
         "bs_plain_stack_device_bytes": (Z, [I, I, I, I]),
         "bs_plain_workspace_bytes": (Z, [I, I, I, I, I]),
         "bs_plain_stack_create": (I, [I, I, I, I, P, Z, P, P, ctypes.POINTER(P)]),
+        "bs_group_workspace_bytes": (Z, [I, P, P, I]),
+        "bs_linear_group": (I, [I, P, P, P, P, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -259,3 +261,25 @@ def bs_plan_budget(order_weight, block_bytes, budget_bytes: int):
     _check(lib.bs_plan_budget(order.size, _ptr(order) if order.size else None, sizes.size, _ptr(sizes),
                               int(budget_bytes), _ptr(out)), "bs_plan_budget")
     return out[:sizes.size]
+
+
+def _handles(handles):
+    return (ctypes.c_void_p * len(handles))(*[int(h) for h in handles])
+
+
+def bs_group_workspace_bytes(handles, n_loaded, batch: int) -> int:
+    counts = np.ascontiguousarray(n_loaded, dtype=np.int32)
+    return int(lib.bs_group_workspace_bytes(len(handles), _handles(handles), _ptr(counts), batch))
+
+
+def bs_linear_group(handles, xs, n_loaded, ys, workspace, stream=None) -> None:
+    """One decode launch over many stacks: ys[l] = xs[l] W_hat_{n_loaded[l]}^T (CUDA
+    tensors, one dtype, batch 1..4)."""
+    nl = len(handles)
+    counts = np.ascontiguousarray(n_loaded, dtype=np.int32)
+    xp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in xs])
+    yp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in ys])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.bs_linear_group(nl, _handles(handles), xp, yp, _ptr(counts), xs[0].shape[0], _dtype_code(xs[0]),
+                             _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "bs_linear_group")

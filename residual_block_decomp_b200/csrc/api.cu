@@ -70,6 +70,43 @@ bool build_factor_maps(bs_stack_s* s) {
 
 bs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BS_OK : BS_ERR_CUDA; }
 
+// The per-linear part of a decode launch, without its workspace pointers.
+void fill_lin(DecodeLin& L, const bs_stack_s* stack, const void* x, void* y, int n_loaded, int batch) {
+  L.blocks = stack->blocks;
+  L.block_bytes = stack->block_bytes;
+  L.x = x;
+  L.y = y;
+  L.inv_s = stack->inv_s;
+  L.m = stack->m;
+  L.d = stack->d;
+  L.n = n_loaded;
+  L.KG = stack->d / kTileCols;
+  L.RT = stack->m / kTileRows;
+  L.NCB = decode_groups_per_block(stack->d, batch);
+  L.seg0 = 0;
+  L.cg0 = 0;
+}
+
+// Workspace of a grouped decode launch: all row-tile counters first (their places
+// depend only on the shapes, so they stay put as the loaded counts change), then each
+// linear's partials.
+struct GroupWs {
+  size_t cnt_bytes, total;
+};
+GroupWs group_ws(int n_linears, const bs_stack_t* stacks, const int* n_loaded, int batch) {
+  GroupWs g{0, 0};
+  for (int l = 0; l < n_linears; ++l) g.cnt_bytes += static_cast<size_t>(stacks[l]->m / kTileRows) * 4;
+  g.cnt_bytes = align_up(g.cnt_bytes, 256);
+  size_t off = g.cnt_bytes;
+  for (int l = 0; l < n_linears; ++l) {
+    const size_t segs = static_cast<size_t>(stacks[l]->m / kTileRows) * n_loaded[l] *
+                        decode_groups_per_block(stacks[l]->d, batch);
+    off = align_up(off + segs * batch * kTileRows * sizeof(float), 256);
+  }
+  g.total = off;
+  return g;
+}
+
 }  // namespace
 
 extern "C" {
@@ -282,28 +319,20 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
 
   if (batch <= kDecodeMaxBatch) {
     if (n_loaded > kDecodeMaxBlocks) return BS_ERR_RANGE;
-    const DecodeWs L = decode_ws_layout(m, d, n_loaded, batch);
-    if (workspace == nullptr || workspace_bytes < L.total) return BS_ERR_CAPACITY;
+    const DecodeWs W = decode_ws_layout(m, d, n_loaded, batch);
+    if (workspace == nullptr || workspace_bytes < W.total) return BS_ERR_CAPACITY;
     if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     DecodeParams p{};
-    p.blocks = stack->blocks;
-    p.block_bytes = stack->block_bytes;
-    p.x = x;
-    p.y = y;
-    p.inv_s = stack->inv_s;
-    p.part = reinterpret_cast<float*>(ws + L.part);
-    p.cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
-    p.err = stack->err;
-    p.m = m;
-    p.d = d;
-    p.n = n_loaded;
-    p.KG = d / kTileCols;
-    p.RT = m / kTileRows;
-    p.NCB = decode_groups_per_block(d, batch);
-    const long long segs = static_cast<long long>(p.RT) * n_loaded * p.NCB;
+    DecodeLin& L = p.lin[0];
+    fill_lin(L, stack, x, y, n_loaded, batch);
+    L.part = reinterpret_cast<float*>(ws + W.part);
+    L.cnt = reinterpret_cast<uint32_t*>(ws + W.cnt);
+    const long long segs = static_cast<long long>(L.RT) * n_loaded * L.NCB;
     if (segs > (1ll << 30)) return BS_ERR_UNSUPPORTED_SHAPE;
+    p.nlin = 1;
     p.segs = static_cast<int>(segs);
+    p.err = stack->err;
     p.x_bf16 = dt == BS_BF16 ? 1 : 0;
     p.inject_unreachable = stack->inject_unreachable;
     stack->inject_unreachable = 0;
@@ -346,6 +375,75 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   const cuuint32_t xbox[2] = {8, static_cast<cuuint32_t>(p.NT)};
   if (!encode(&tm_x, dt == BS_BF16, 2, const_cast<void*>(x), xdims, xstr, xbox)) return BS_ERR_CUDA;
   return cuda_status(launch_prefill(p, tm_x, stack->tm_u, stack->tm_v, dt == BS_BF16 ? 1 : 0, stream));
+}
+
+size_t bs_group_workspace_bytes(int n_linears, const bs_stack_t* stacks, const int* n_loaded, int batch) {
+  if (n_linears <= 0 || n_linears > kDecodeGroupMax || stacks == nullptr || n_loaded == nullptr || batch <= 0 ||
+      batch > kDecodeMaxBatch)
+    return 0;
+  for (int l = 0; l < n_linears; ++l)
+    if (stacks[l] == nullptr || stacks[l]->plain || n_loaded[l] < 0) return 0;
+  return group_ws(n_linears, stacks, n_loaded, batch).total;
+}
+
+bs_status bs_linear_group(int n_linears, const bs_stack_t* stacks, const void* const* x, void* const* y,
+                          const int* n_loaded, int batch, bs_dtype dt, void* workspace, size_t workspace_bytes,
+                          bs_stream_t stream) {
+  if (n_linears <= 0 || n_linears > kDecodeGroupMax || stacks == nullptr || x == nullptr || y == nullptr ||
+      n_loaded == nullptr || batch <= 0 || batch > kDecodeMaxBatch)
+    return BS_ERR_INVALID_ARG;
+  if (dt != BS_F16 && dt != BS_BF16) return BS_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BS_ERR_NO_DEVICE;
+  for (int l = 0; l < n_linears; ++l) {
+    const bs_stack_s* st = stacks[l];
+    if (st == nullptr || st->plain || x[l] == nullptr || y[l] == nullptr || st->device != dev) return BS_ERR_INVALID_ARG;
+    if (n_loaded[l] < 0 || n_loaded[l] > st->n_blocks || n_loaded[l] > kDecodeMaxBlocks) return BS_ERR_RANGE;
+    if (!aligned(x[l], 16) || !aligned(y[l], 16)) return BS_ERR_ALIGNMENT;
+  }
+  const GroupWs W = group_ws(n_linears, stacks, n_loaded, batch);
+  if (workspace == nullptr || workspace_bytes < W.total) return BS_ERR_CAPACITY;
+  if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // the table is ~22 KB: keep it off the thread's stack
+  static thread_local DecodeGroupParams p;
+  p = DecodeGroupParams{};
+  size_t cnt_off = 0, part_off = W.cnt_bytes;
+  long long segs = 0;
+  int cgs = 0, nlin = 0;
+  for (int l = 0; l < n_linears; ++l) {
+    const bs_stack_s* st = stacks[l];
+    const size_t RT = static_cast<size_t>(st->m / kTileRows);
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + cnt_off);
+    cnt_off += RT * 4;
+    if (n_loaded[l] == 0) {   // no blocks: y is zero
+      const cudaError_t e = cudaMemsetAsync(y[l], 0, static_cast<size_t>(batch) * st->m * 2, stream);
+      if (e != cudaSuccess) return BS_ERR_CUDA;
+      continue;
+    }
+    DecodeLin& L = p.lin[nlin++];
+    fill_lin(L, st, x[l], y[l], n_loaded[l], batch);
+    L.cnt = cnt;
+    L.part = reinterpret_cast<float*>(ws + part_off);
+    const long long ls = static_cast<long long>(L.RT) * L.n * L.NCB;
+    part_off = align_up(part_off + static_cast<size_t>(ls) * batch * kTileRows * sizeof(float), 256);
+    L.seg0 = static_cast<int>(segs);
+    L.cg0 = cgs;
+    segs += ls;
+    cgs += L.n * L.NCB;
+    if (segs > (1ll << 30)) return BS_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (nlin == 0) return BS_OK;
+  p.nlin = nlin;
+  p.segs = static_cast<int>(segs);
+  p.err = stacks[0]->err;
+  p.x_bf16 = dt == BS_BF16 ? 1 : 0;
+  p.inject_unreachable = 0;
+  p.timeout_ns = stacks[0]->timeout_ns;
+  const int slack = stacks[0]->sm_count > 32 ? 4 : 0;
+  const int ctas = stacks[0]->sm_count - slack;
+  const int grid = segs < ctas ? static_cast<int>(segs) : ctas;
+  return cuda_status(launch_decode_group(p, batch, grid, stream));
 }
 
 bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_stream_t stream) {

@@ -131,39 +131,89 @@ static_assert(sizeof(Ctl) <= 8192, "control block");
 struct Seg {
   int i, rt, kgA, len, cg;
   int cgb;   // chunk group within block i
+  int l;     // linear of the launch
+  int sl;    // segment within linear l
 };
-__device__ __forceinline__ Seg seg_of(int s, const DecodeParams& p, int C) {
+// Linear l of a launch (the last one for an index past the end, which walks reach only
+// after their last segment).
+template <int G>
+__device__ __forceinline__ const DecodeLin& lin_at(const DecodeArgs<G>& p, int l) {
+  return p.lin[G == 1 ? 0 : (l < p.nlin ? l : p.nlin - 1)];
+}
+// The linear holding global segment s: the last one whose first segment is <= s.
+template <int G>
+__device__ __forceinline__ int lin_of_seg(const DecodeArgs<G>& p, int s) {
+  if (G == 1) return 0;
+  int lo = 0, hi = p.nlin - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.lin[mid].seg0 <= s) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+template <int G>
+__device__ __forceinline__ Seg seg_of(int s, const DecodeArgs<G>& p, int C) {
   Seg g;
-  g.cg = s / p.RT;
-  g.rt = s - g.cg * p.RT;
-  g.i = g.cg / p.NCB;
-  g.cgb = g.cg - g.i * p.NCB;
+  g.l = lin_of_seg(p, s);
+  const DecodeLin& L = lin_at(p, g.l);
+  g.sl = s - L.seg0;
+  g.cg = g.sl / L.RT;
+  g.rt = g.sl - g.cg * L.RT;
+  g.i = g.cg / L.NCB;
+  g.cgb = g.cg - g.i * L.NCB;
   g.kgA = g.cgb * C;
-  g.len = min(C, p.KG - g.kgA);
+  g.len = min(C, L.KG - g.kgA);
   return g;
 }
-// The segment after g (chunk-group-major numbering), without divisions.
-__device__ __forceinline__ void seg_next(Seg& g, const DecodeParams& p, int C) {
-  if (++g.rt == p.RT) {
+// The segment after g (chunk-group-major within a linear, linears one after another),
+// without divisions.
+template <int G>
+__device__ __forceinline__ void seg_next(Seg& g, const DecodeArgs<G>& p, int C) {
+  ++g.sl;
+  const DecodeLin& L = lin_at(p, g.l);
+  if (++g.rt == L.RT) {
     g.rt = 0;
     ++g.cg;
-    if (++g.cgb == p.NCB) {
+    if (++g.cgb == L.NCB) {
       g.cgb = 0;
       ++g.i;
+      if (G > 1 && g.i == L.n) {   // on to the next linear (each has at least one block)
+        ++g.l;
+        g.i = 0;
+        g.cg = 0;
+        g.sl = 0;
+      }
     }
     g.kgA = g.cgb * C;
-    g.len = min(C, p.KG - g.kgA);
+    g.len = min(C, lin_at(p, g.l).KG - g.kgA);
   }
 }
+// Chunk group cg of linear l, and the one after it.
+struct GroupRef {
+  int l, cg;
+};
+template <int G>
+__device__ __forceinline__ GroupRef group_next(GroupRef r, const DecodeArgs<G>& p) {
+  const DecodeLin& L = lin_at(p, r.l);
+  if (++r.cg == L.n * L.NCB && G > 1) {
+    ++r.l;
+    r.cg = 0;
+  }
+  return r;
+}
 
-// The run of segments [s0, s1) of CTA `cta`.  With at most as many chunk groups as CTAs,
-// every group gets floor or ceil(grid / groups) CTAs and splits its RT segments evenly
-// among them, so no CTA spans two groups (building a group's activation set is paid
-// once per CTA); otherwise the segments are split contiguously and a CTA spans several
-// groups, whose sets after the first are built in the background.
-__device__ __forceinline__ void cta_range(const DecodeParams& p, int cta, int grid, int& s0, int& s1) {
-  const int NG = p.n * p.NCB;
-  if (NG <= grid) {
+// The run of segments [s0, s1) of CTA `cta`.  For one linear with at most as many chunk
+// groups as CTAs, every group gets floor or ceil(grid / groups) CTAs and splits its RT
+// segments evenly among them, so no CTA spans two groups (building a group's activation
+// set is paid once per CTA); otherwise (more groups, or several linears) the segments
+// are split contiguously and a CTA spans several groups, whose sets after the first
+// are built in the background.
+template <int G>
+__device__ __forceinline__ void cta_range(const DecodeArgs<G>& p, int cta, int grid, int& s0, int& s1) {
+  const DecodeLin& L = p.lin[0];
+  const int NG = L.n * L.NCB;
+  if (G == 1 && NG <= grid) {
     const int base = grid / NG, extra = grid - base * NG;
     int g, w, k;
     if (cta < extra * (base + 1)) {
@@ -176,8 +226,8 @@ __device__ __forceinline__ void cta_range(const DecodeParams& p, int cta, int gr
       w = c2 - (g - extra) * base;
       k = base;
     }
-    s0 = g * p.RT + (w * p.RT) / k;
-    s1 = g * p.RT + ((w + 1) * p.RT) / k;
+    s0 = g * L.RT + (w * L.RT) / k;
+    s1 = g * L.RT + ((w + 1) * L.RT) / k;
   } else {
     s0 = static_cast<int>(static_cast<long long>(cta) * p.segs / grid);
     s1 = static_cast<int>(static_cast<long long>(cta + 1) * p.segs / grid);
@@ -192,18 +242,19 @@ __device__ __forceinline__ float x_at(const void* x, int bf16, size_t idx) {
   const uint16_t h = static_cast<const uint16_t*>(x)[idx];
   return bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
 }
-__device__ __forceinline__ void set_error(const DecodeParams& p, Ctl* ctl) {
+template <int G>
+__device__ __forceinline__ void set_error(const DecodeArgs<G>& p, Ctl* ctl) {
   ctl->abort = 1;
   atomicOr(p.err, kErrTimeout);
 }
 
 // Byte offsets inside one block record.
-__device__ __forceinline__ const uint8_t* record(const DecodeParams& p, int i) {
-  return p.blocks + static_cast<size_t>(i) * p.block_bytes;
+__device__ __forceinline__ const uint8_t* record(const DecodeLin& L, int i) {
+  return L.blocks + static_cast<size_t>(i) * L.block_bytes;
 }
-__device__ __forceinline__ size_t u_offset(const DecodeParams& p) { return static_cast<size_t>(p.m) * p.d / 8; }
-__device__ __forceinline__ size_t v_offset(const DecodeParams& p) {
-  return u_offset(p) + static_cast<size_t>(2) * kK * p.m;
+__device__ __forceinline__ size_t u_offset(const DecodeLin& L) { return static_cast<size_t>(L.m) * L.d / 8; }
+__device__ __forceinline__ size_t v_offset(const DecodeLin& L) {
+  return u_offset(L) + static_cast<size_t>(2) * kK * L.m;
 }
 
 // K-step t of a unit from one sign word: bit t of every byte moved to bit 7 and the
@@ -280,12 +331,12 @@ __device__ __forceinline__ void v_row(const uint8_t* row, float (&v)[16]) {
 struct Group {
   int i, col0, gcols;
 };
-__device__ __forceinline__ Group group_of(const DecodeParams& p, int cg, int C) {
+__device__ __forceinline__ Group group_of(const DecodeLin& L, int cg, int C) {
   Group g;
-  g.i = cg / p.NCB;
-  const int k0 = (cg - g.i * p.NCB) * C;
+  g.i = cg / L.NCB;
+  const int k0 = (cg - g.i * L.NCB) * C;
   g.col0 = k0 * kTileCols;
-  g.gcols = min(C, p.KG - k0) * kTileCols;
+  g.gcols = min(C, L.KG - k0) * kTileCols;
   return g;
 }
 
@@ -307,15 +358,15 @@ struct SetSrc {
 //              as the two int8 planes q = 256 hi + lo, and the integer sums of q;
 // with ctl->{amax, csum, sig}[slot] as the shared state.  Per-column maxima and sums
 // are warp reduce-scatters and one shared atomic per column and warp.
-template <bool kGlobal>
-__device__ __forceinline__ float x_scaled(const DecodeParams& p, const SetSrc& S, int c, int b) {
+template <bool kGlobal, typename P>
+__device__ __forceinline__ float x_scaled(const P& p, const SetSrc& S, int c, int b) {
   const uint16_t h = S.x[b * S.xs + c];
   const float xv = p.x_bf16 ? __uint_as_float(static_cast<uint32_t>(h) << 16) : __half2float(__ushort_as_half(h));
   return __fmul_rn(xv, kGlobal ? __ldg(S.is + c) : S.is[c]);
 }
 
-template <int B, bool kGlobal>
-__device__ void set_max(const DecodeParams& p, Ctl* ctl, int slot, const SetSrc& S, int gcols, int zt, int NT) {
+template <int B, bool kGlobal, typename P>
+__device__ void set_max(const P& p, Ctl* ctl, int slot, const SetSrc& S, int gcols, int zt, int NT) {
   const int lane = zt & 31;
 #pragma unroll
   for (int b = 0; b < B; ++b) {
@@ -334,8 +385,8 @@ __device__ void set_max(const DecodeParams& p, Ctl* ctl, int slot, const SetSrc&
   }
 }
 
-template <int B, bool kGlobal>
-__device__ void set_quant(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
+template <int B, bool kGlobal, typename P>
+__device__ void set_quant(const P& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
                           int NT) {
   using K = Cfg<B>;
   constexpr int NB = K::NB, NCOL = K::NCOL;
@@ -376,8 +427,8 @@ __device__ void set_quant(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* se
   }
 }
 
-template <int B, bool kGlobal>
-__device__ void build_set(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
+template <int B, bool kGlobal, typename P>
+__device__ void build_set(const P& p, Ctl* ctl, int slot, uint8_t* set, const SetSrc& S, int gcols, int zt,
                           int NT, int bar) {
   constexpr int NCOL = Cfg<B>::NCOL;
   const int nw = NT >> 5;
@@ -409,16 +460,17 @@ __device__ void build_set(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* se
 }
 
 // A set built from global memory (the epilogue warps, in the background).
-template <int B>
-__device__ void build_set_global(const DecodeParams& p, Ctl* ctl, int slot, uint8_t* set, int cg, int zt, int NT,
-                                 int bar) {
-  const Group G = group_of(p, cg, Cfg<B>::C);
+template <int B, int G>
+__device__ void build_set_global(const DecodeArgs<G>& p, Ctl* ctl, int slot, uint8_t* set, GroupRef gr, int zt,
+                                 int NT, int bar) {
+  const DecodeLin& L = lin_at(p, gr.l);
+  const Group g = group_of(L, gr.cg, Cfg<B>::C);
   SetSrc S;
-  S.v = record(p, G.i) + v_offset(p) + static_cast<size_t>(G.col0) * 32;
-  S.x = static_cast<const uint16_t*>(p.x) + G.col0;
-  S.is = p.inv_s + G.col0;
-  S.xs = p.d;
-  build_set<B, true>(p, ctl, slot, set, S, G.gcols, zt, NT, bar);
+  S.v = record(L, g.i) + v_offset(L) + static_cast<size_t>(g.col0) * 32;
+  S.x = static_cast<const uint16_t*>(L.x) + g.col0;
+  S.is = L.inv_s + g.col0;
+  S.xs = L.d;
+  build_set<B, true>(p, ctl, slot, set, S, g.gcols, zt, NT, bar);
 }
 
 // MMA issued by the elected lane of a warp whose lanes hold the same operands.
@@ -438,8 +490,8 @@ __device__ __forceinline__ void commit_elect(uint64_t* bar) {
       : "memory");
 }
 
-template <int B>
-__global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const DecodeParams p) {
+template <int B, int G>
+__global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const __grid_constant__ DecodeArgs<G> p) {
   using K = Cfg<B>;
   constexpr int NB = K::NB, NCOL = K::NCOL, C = K::C, NS = K::NS, T = K::T, NACC = K::NACC;
   constexpr uint32_t IDESC = make_idesc(2u, 1u, 1u, 128u, NB);   // s32 <- s8 x s8, M = 128, N = NB
@@ -459,8 +511,10 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
   const int nseg = s1 - s0;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
   const Seg sg0 = seg_of(s0, p, C);
-  const int last_cg = seg_of(s1 - 1, p, C).cg;
-  const int NZ = last_cg - sg0.cg + 1;               // chunk groups this CTA touches (consecutive)
+  const Seg sgz = seg_of(s1 - 1, p, C);
+  // chunk groups this CTA touches (consecutive in the launch's numbering)
+  const int NZ = (lin_at(p, sgz.l).cg0 + sgz.cg) - (lin_at(p, sg0.l).cg0 + sg0.cg) + 1;
+  const DecodeLin& L0 = lin_at(p, sg0.l);            // the linear of the first segment
 
   griddep_launch_dependents();
 
@@ -506,20 +560,21 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       const int st = jj % NS;
       const uint32_t bytes = static_cast<uint32_t>(sg.len) * kTileBytes;
       mbar_arrive_expect_tx(&ctl->sfull[st], bytes);
+      const DecodeLin& L = lin_at(p, sg.l);
       bulk_g2s(stages + st * K::STAGE,
-               record(p, sg.i) + (static_cast<size_t>(sg.rt) * p.KG + sg.kgA) * kTileBytes, bytes, &ctl->sfull[st]);
+               record(L, sg.i) + (static_cast<size_t>(sg.rt) * L.KG + sg.kgA) * kTileBytes, bytes, &ctl->sfull[st]);
     };
     // The first group's V rows (into the second set slot) and 1/s, and the first stages:
     // stack memory and the scale vector, read before the previous kernel has finished.
     // (Timeout test: CTA 0 leaves out its first stage, so its waits run out while the
     // other CTAs complete and count their partials.)
-    const Group G0 = group_of(p, sg0.cg, C);
+    const Group G0 = group_of(L0, sg0.cg, C);
     const int first = min(NS, nseg);
     if (lane == 31) {
       mbar_arrive_expect_tx(&ctl->vstage, static_cast<uint32_t>(G0.gcols) * 36u);
-      bulk_g2s(sets + K::SET, record(p, G0.i) + v_offset(p) + static_cast<size_t>(G0.col0) * 32,
+      bulk_g2s(sets + K::SET, record(L0, G0.i) + v_offset(L0) + static_cast<size_t>(G0.col0) * 32,
                static_cast<uint32_t>(G0.gcols) * 32u, &ctl->vstage);
-      bulk_g2s(stg + B * C * kTileCols * 2, p.inv_s + G0.col0, static_cast<uint32_t>(G0.gcols) * 4u, &ctl->vstage);
+      bulk_g2s(stg + B * C * kTileCols * 2, L0.inv_s + G0.col0, static_cast<uint32_t>(G0.gcols) * 4u, &ctl->vstage);
     }
     if (lane < first && !(skip_first && lane == 0)) issue_stage(lane, seg_of(s0 + lane, p, C));
     // x only after the kernel ahead has finished (it may have written x)
@@ -527,7 +582,7 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
     if (lane == 0) mbar_arrive_expect_tx(&ctl->xstage, static_cast<uint32_t>(B * G0.gcols) * 2u);
     __syncwarp();
     if (lane < B)
-      bulk_g2s(stg + lane * C * kTileCols * 2, static_cast<const uint16_t*>(p.x) + static_cast<size_t>(lane) * p.d + G0.col0,
+      bulk_g2s(stg + lane * C * kTileCols * 2, static_cast<const uint16_t*>(L0.x) + static_cast<size_t>(lane) * L0.d + G0.col0,
                static_cast<uint32_t>(G0.gcols) * 2u, &ctl->xstage);
     if (lane == 0) {
       Seg sc = seg_of(s0 + first, p, C);   // the segment of the next stage to issue
@@ -556,15 +611,17 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       // warm L2 with the V rows of the second group (stack memory, read before the kernel
       // ahead has finished); the first group's inputs arrive in shared memory
       if (NZ > 1) {
-        const Group G = group_of(p, sg0.cg + 1, C);
-        for (int c = zt; c < G.gcols; c += K::ZTHREADS)
-          prefetch_l2(record(p, G.i) + v_offset(p) + static_cast<size_t>(G.col0 + c) * 32);
+        const GroupRef g1 = group_next(GroupRef{sg0.l, sg0.cg}, p);
+        const DecodeLin& L1 = lin_at(p, g1.l);
+        const Group G1 = group_of(L1, g1.cg, C);
+        for (int c = zt; c < G1.gcols; c += K::ZTHREADS)
+          prefetch_l2(record(L1, G1.i) + v_offset(L1) + static_cast<size_t>(G1.col0 + c) * 32);
       }
       griddep_wait();   // the workspace, y and x belong to this launch only from here on
       bool ok = mbar_wait(&ctl->vstage, 0, deadline, abort_flag);
       ok = ok && mbar_wait(&ctl->xstage, 0, deadline, abort_flag);
       if (!ok) set_error(p, ctl);   // the set is then garbage; every later wait sees the abort flag
-      const Group G0 = group_of(p, sg0.cg, C);
+      const Group G0 = group_of(L0, sg0.cg, C);
       SetSrc S;
       S.v = sets + K::SET;
       S.x = reinterpret_cast<const uint16_t*>(stg);
@@ -670,9 +727,9 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
         if (++c == sg.len) {
           c = 0;
           ++j;
-          const int cg = sg.cg;
+          const int cg = sg.cg, l = sg.l;
           seg_next(sg, p, C);
-          if (sg.cg != cg) ++zk;
+          if (sg.cg != cg || sg.l != l) ++zk;
         }
       }
       if (!ok) set_error(p, ctl);
@@ -686,7 +743,6 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       const int et = threadIdx.x - 32 * K::WEPI;                   // 0 .. 127
       const int tid = 32 * q + lane;                               // row of the tile = TMEM lane
       const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-      const int NC = p.n * p.NCB;                                  // partials per row tile
       uint32_t zr[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) zr[e] = 0u;
@@ -701,7 +757,7 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       // the CTA's second chunk group (if any) is built here, while the teams and issuers
       // work through the first
       if (NZ > 1) {
-        build_set_global<B>(p, ctl, 1, sets + K::SET, sg0.cg + 1, et, 128, kBarEpi);
+        build_set_global<B>(p, ctl, 1, sets + K::SET, group_next(GroupRef{sg0.l, sg0.cg}, p), et, 128, kBarEpi);
         if (et == 0) mbar_arrive(&ctl->zready[1]);
       }
       bool failed = false;
@@ -709,7 +765,8 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       Seg sg = sg0;
       for (int j = 0; j < nseg; ++j, seg_next(sg, p, C)) {
         const int a = j % NACC;
-        const uint4* urow = reinterpret_cast<const uint4*>(record(p, sg.i) + u_offset(p) +
+        const DecodeLin& L = lin_at(p, sg.l);
+        const uint4* urow = reinterpret_cast<const uint4*>(record(L, sg.i) + u_offset(L) +
                                                            static_cast<size_t>(sg.rt * kTileRows + tid) * kK * 2);
         const uint4 ua = __ldg(urow), ub = __ldg(urow + 1);
         bool ok = !failed && mbar_wait(&ctl->accfull[a], static_cast<uint32_t>((j / NACC) & 1), deadline, abort_flag);
@@ -748,21 +805,22 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->acc_free[a]);
-          float* dst = p.part + static_cast<size_t>(s0 + j) * B * kTileRows;
+          float* dst = L.part + static_cast<size_t>(sg.sl) * B * kTileRows;
 #pragma unroll
           for (int b = 0; b < B; ++b) dst[b * kTileRows + tid] = part[b];
         } else {
           set_error(p, ctl);
           failed = true;   // keep walking: every warp must pass the same barriers below
         }
-        const bool group_end = (j + 1 == nseg) || sg.rt + 1 == p.RT;
+        const bool group_end = (j + 1 == nseg) || sg.rt + 1 == L.RT;
         if (group_end) {
           // this group's set and its sig / csum are no longer read: build group zk + 2
           // (if the CTA has one) into the same slot
           if (bar_any(kBarEpi, 128, failed || *abort_flag != 0)) {
             failed = true;
           } else if (zk + 2 < NZ) {
-            build_set_global<B>(p, ctl, zk & 1, sets + (zk & 1) * K::SET, sg.cg + 2, et, 128, kBarEpi);
+            build_set_global<B>(p, ctl, zk & 1, sets + (zk & 1) * K::SET,
+                                group_next(group_next(GroupRef{sg.l, sg.cg}, p), p), et, 128, kBarEpi);
             if (et == 0) mbar_arrive(&ctl->zready[zk & 1]);
           }
           ++zk;
@@ -785,19 +843,19 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
   __syncthreads();
   if (ctl->count_ok) {
     constexpr int KS = K::THREADS / kTileRows;   // slices per row tile
-    const int NC = p.n * p.NCB;                  // partials per row tile
     const int r = threadIdx.x % kTileRows, ks = threadIdx.x / kTileRows;
     // the sign stages are drained by now: [4 tiles][KS][B][128] slice sums, then the row
-    // tiles this CTA completed in the current round
+    // tiles (linear << 16 | row tile) this CTA completed in the current round
     float* red = reinterpret_cast<float*>(stages);
     int* red_rt = reinterpret_cast<int*>(stages + 4 * KS * B * kTileRows * 4);
     for (int base = 0; base < nseg; base += K::THREADS) {
       const int e = base + static_cast<int>(threadIdx.x);
       if (e < nseg) {
-        const int rt = (s0 + e) % p.RT;
-        if (atomicAdd(p.cnt + rt, 1u) == static_cast<uint32_t>(NC - 1)) {
+        const Seg se = seg_of(s0 + e, p, C);
+        const DecodeLin& L = lin_at(p, se.l);
+        if (atomicAdd(L.cnt + se.rt, 1u) == static_cast<uint32_t>(L.n * L.NCB - 1)) {
           const int idx = atomicAdd(&ctl->nred, 1);
-          red_rt[idx] = rt;
+          red_rt[idx] = (se.l << 16) | se.rt;
         }
       }
       __syncthreads();
@@ -808,23 +866,34 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
       for (int q0 = 0; q0 < nred; q0 += kTB) {
         const int nq = min(kTB, nred - q0);
         if (ks < KS) {
-          const size_t stride = static_cast<size_t>(p.RT) * B * kTileRows;
+          const float* pp[kTB];
+          size_t stride[kTB];
+          int nc[kTB];
+          int ncmax = 0;
+#pragma unroll
+          for (int t = 0; t < kTB; ++t) {
+            const int code = t < nq ? red_rt[q0 + t] : red_rt[q0];
+            const DecodeLin& L = lin_at(p, code >> 16);
+            pp[t] = L.part + static_cast<size_t>(code & 0xffff) * B * kTileRows + r;
+            stride[t] = static_cast<size_t>(L.RT) * B * kTileRows;
+            nc[t] = t < nq ? L.n * L.NCB : 0;   // partials of the row tile
+            ncmax = max(ncmax, nc[t]);
+          }
           float acc[kTB][B];
 #pragma unroll
           for (int t = 0; t < kTB; ++t)
 #pragma unroll
             for (int b = 0; b < B; ++b) acc[t][b] = 0.0f;
-          for (int c0 = ks; c0 < NC; c0 += 4 * KS) {
+          for (int c0 = ks; c0 < ncmax; c0 += 4 * KS) {
             float v[kTB][4][B];
 #pragma unroll
             for (int t = 0; t < kTB; ++t) {
-              const float* pp = p.part + static_cast<size_t>(t < nq ? red_rt[q0 + t] : 0) * B * kTileRows + r;
 #pragma unroll
               for (int e2 = 0; e2 < 4; ++e2)
 #pragma unroll
                 for (int b = 0; b < B; ++b) {
                   const int cg = c0 + e2 * KS;
-                  v[t][e2][b] = (t < nq && cg < NC) ? __ldcg(pp + cg * stride + b * kTileRows) : 0.0f;
+                  v[t][e2][b] = cg < nc[t] ? __ldcg(pp[t] + cg * stride[t] + b * kTileRows) : 0.0f;
                 }
             }
 #pragma unroll
@@ -842,14 +911,15 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
         __syncthreads();
         for (int idx = threadIdx.x; idx < nq * kTileRows; idx += K::THREADS) {
           const int t = idx / kTileRows, rr = idx - t * kTileRows;
-          const int rt = red_rt[q0 + t];
+          const int code = red_rt[q0 + t], rt = code & 0xffff;
+          const DecodeLin& L = lin_at(p, code >> 16);
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             float sum = 0.0f;
             for (int k = 0; k < KS; ++k) sum += red[((t * KS + k) * B + b) * kTileRows + rr];
-            store_y(p.y, p.x_bf16, static_cast<size_t>(b) * p.m + static_cast<size_t>(rt) * kTileRows + rr, sum);
+            store_y(L.y, p.x_bf16, static_cast<size_t>(b) * L.m + static_cast<size_t>(rt) * kTileRows + rr, sum);
           }
-          if (rr == 0) p.cnt[rt] = 0u;   // the next call starts from zero
+          if (rr == 0) L.cnt[rt] = 0u;   // the next call starts from zero
         }
         __syncthreads();
       }
@@ -864,10 +934,10 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const Decode
   }
 }
 
-template <int B>
-cudaError_t launch_b(const DecodeParams& p, int grid, cudaStream_t stream) {
+template <int B, int G>
+cudaError_t launch_b(const DecodeArgs<G>& p, int grid, cudaStream_t stream) {
   using K = Cfg<B>;
-  auto kern = decode_kernel<B>;
+  auto kern = decode_kernel<B, G>;
   static bool configured[64] = {};   // the attribute is set once per device, outside any capture
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -905,10 +975,20 @@ size_t decode_smem_bytes(int batch) {
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream) {
   switch (batch) {
-    case 1: return launch_b<1>(p, grid, stream);
-    case 2: return launch_b<2>(p, grid, stream);
-    case 3: return launch_b<3>(p, grid, stream);
-    case 4: return launch_b<4>(p, grid, stream);
+    case 1: return launch_b<1, 1>(p, grid, stream);
+    case 2: return launch_b<2, 1>(p, grid, stream);
+    case 3: return launch_b<3, 1>(p, grid, stream);
+    case 4: return launch_b<4, 1>(p, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode_group(const DecodeGroupParams& p, int batch, int grid, cudaStream_t stream) {
+  switch (batch) {
+    case 1: return launch_b<1, kDecodeGroupMax>(p, grid, stream);
+    case 2: return launch_b<2, kDecodeGroupMax>(p, grid, stream);
+    case 3: return launch_b<3, kDecodeGroupMax>(p, grid, stream);
+    case 4: return launch_b<4, kDecodeGroupMax>(p, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }

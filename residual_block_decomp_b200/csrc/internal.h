@@ -52,22 +52,34 @@ inline DecodeWs decode_ws_layout(int m, int d, int n, int batch) {
   return w;
 }
 
-struct DecodeParams {
+// One linear of a decode launch.  Segments of all linears of a launch are numbered
+// linear after linear (seg0 = the first segment of this linear, cg0 its first chunk group).
+struct DecodeLin {
   const uint8_t* blocks;       // record i at blocks + i * block_bytes
   unsigned long long block_bytes;
   const void* x;               // batch x d, f16 or bf16
   void* y;                     // batch x m, same dtype
   const float* inv_s;          // d
-  float* part;                 // [segs][batch][128] partial outputs of the segments
+  float* part;                 // [segments of this linear][batch][128] partial outputs
   uint32_t* cnt;               // [RT] partials of the row tile that have arrived
-  uint32_t* err;               // sticky device error word
   int m, d, n, KG, RT, NCB;    // NCB chunk groups per block
-  int segs;                    // RT * n * NCB
+  int seg0, cg0;
+};
+// A decode launch over G linears at most (kernel parameter block: one linear for
+// bs_linear, up to kDecodeGroupMax for bs_linear_group).
+constexpr int kDecodeGroupMax = 256;
+template <int G>
+struct DecodeArgs {
+  DecodeLin lin[G];
+  int nlin;                    // linears in use, each with at least one segment
+  int segs;                    // segments of all linears
+  uint32_t* err;               // sticky device error word
   int x_bf16;
   int inject_unreachable;      // CTA 0's first sign copy is never issued (timeout test)
   unsigned long long timeout_ns;
 };
-
+using DecodeParams = DecodeArgs<1>;
+using DecodeGroupParams = DecodeArgs<kDecodeGroupMax>;
 struct PrefillParams {
   const uint8_t* blocks;
   unsigned long long block_bytes;
@@ -108,6 +120,7 @@ cudaError_t launch_plain_reconstruct(const uint8_t* blocks, unsigned long long b
 // Launchers (decode.cu, prefill.cu, aux_kernels.cu).  They return cudaSuccess or the
 // launch error.
 cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream);
+cudaError_t launch_decode_group(const DecodeGroupParams& p, int batch, int grid, cudaStream_t stream);
 size_t decode_smem_bytes(int batch);
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_u,

@@ -54,6 +54,14 @@ class BitStackLinear:
         self.host_records.append(pinned)
         return len(self.host_records) - 1
 
+    def add_pinned_record(self, pinned: torch.Tensor) -> int:
+        """Keeps an already pinned record (uint8, bs_block_bytes long) without copying
+        it; several stacks may share one storage copy."""
+        if pinned.numel() != self.block_bytes or not pinned.is_pinned():
+            raise ValueError("need a pinned record of the stack's block size")
+        self.host_records.append(pinned)
+        return len(self.host_records) - 1
+
     # ----------------------------------------------------------- memory side -----
     @property
     def n_blocks(self) -> int:

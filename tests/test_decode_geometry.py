@@ -217,3 +217,137 @@ def test_expansion_rule_reads_columns_in_order():
                     a = ((w >> t) & 0x01010101).astype("<u4").view(np.uint8)   # bytes (pw, q)
                     cols = kg * 256 + 32 * t + np.arange(32)
                     assert np.array_equal(a.astype(bool), neg[rt * 128 + r, cols])
+
+
+# ------------------------------------------------------------ grouped launches -----
+class Lin:
+    def __init__(self, m, d, n, b, seg0, cg0):
+        K = Cfg(b)
+        self.m, self.d, self.n = m, d, n
+        self.RT, self.KG = m // 128, d // 256
+        self.NCB = -(-self.KG // K.C)
+        self.seg0, self.cg0 = seg0, cg0
+        self.segs = self.RT * n * self.NCB
+
+
+def group_table(shapes, b):
+    """The host's table: linears with blocks, segments and chunk groups numbered one
+    linear after another (bs_linear_group)."""
+    tab, seg, cg = [], 0, 0
+    for (m, d, n) in shapes:
+        if n == 0:
+            continue
+        L = Lin(m, d, n, b, seg, cg)
+        tab.append(L)
+        seg += L.segs
+        cg += n * L.NCB
+    return tab, seg
+
+
+def seg_of(tab, s, C):
+    """Mirror of the kernel's seg_of: the last linear whose first segment is <= s."""
+    lo, hi = 0, len(tab) - 1
+    while lo < hi:
+        mid = (lo + hi + 1) >> 1
+        if tab[mid].seg0 <= s:
+            lo = mid
+        else:
+            hi = mid - 1
+    L = tab[lo]
+    sl = s - L.seg0
+    cg, rt = divmod(sl, L.RT)
+    i, cgb = divmod(cg, L.NCB)
+    return dict(l=lo, sl=sl, cg=cg, rt=rt, i=i, cgb=cgb, kgA=cgb * C, len=min(C, L.KG - cgb * C))
+
+
+def seg_next(tab, g, C):
+    """Mirror of the kernel's seg_next (no divisions, linears one after another)."""
+    g = dict(g)
+    g["sl"] += 1
+    L = tab[min(g["l"], len(tab) - 1)]
+    g["rt"] += 1
+    if g["rt"] == L.RT:
+        g["rt"] = 0
+        g["cg"] += 1
+        g["cgb"] += 1
+        if g["cgb"] == L.NCB:
+            g["cgb"] = 0
+            g["i"] += 1
+            if g["i"] == L.n:
+                g["l"] += 1
+                g["i"] = g["cg"] = g["sl"] = 0
+        g["kgA"] = g["cgb"] * C
+        g["len"] = min(C, tab[min(g["l"], len(tab) - 1)].KG - g["kgA"])
+    return g
+
+
+def group_next(tab, l, cg):
+    L = tab[min(l, len(tab) - 1)]
+    cg += 1
+    if cg == L.n * L.NCB:
+        return l + 1, 0
+    return l, cg
+
+
+def _model(counts, layers=2):
+    from workloads import LLAMA3_8B_LINEARS
+    shapes = [(m, d) for _ in range(layers) for (_, m, d) in LLAMA3_8B_LINEARS]
+    return [(m, d, counts[j % len(counts)]) for j, (m, d) in enumerate(shapes)]
+
+
+GROUPS = [_model([3, 0, 1, 5, 2, 16, 4]), _model([1]), _model([16, 2, 0, 0, 9, 1, 3], layers=4),
+          [(128, 256, 1), (256, 512, 2), (128, 256, 0), (1024, 4096, 3)]]
+
+
+@pytest.mark.parametrize("gi", range(len(GROUPS)))
+@pytest.mark.parametrize("b", [1, 3])
+def test_grouped_walk_covers_every_linear_once_and_stays_in_bounds(gi, b):
+    """A grouped launch: every unit of every linear with blocks is covered exactly once;
+    the walk (seg_next) agrees with a fresh lookup (seg_of) at every step; each sign
+    copy, V and U read and partial write lies inside its own linear's areas; a CTA's
+    chunk groups are consecutive in the launch's numbering, and the background set
+    builds (group_next) name exactly the groups the walk reaches."""
+    K = Cfg(b)
+    shapes = GROUPS[gi]
+    tab, segs = group_table(shapes, b)
+    grid = min(SMS - 4, segs)
+    seen = set()
+    for cta in range(grid):
+        s0, s1 = cta * segs // grid, (cta + 1) * segs // grid
+        assert s1 > s0
+        g = seg_of(tab, s0, K.C)
+        gids = []
+        for s in range(s0, s1):
+            f = seg_of(tab, s, K.C)
+            assert g == f, (cta, s, g, f)
+            L = tab[g["l"]]
+            assert 0 <= g["i"] < L.n and 1 <= g["len"] <= K.C and g["sl"] == s - L.seg0
+            assert (g["rt"] * L.KG + g["kgA"]) * 4096 + g["len"] * 4096 <= L.m * L.d // 8
+            assert (g["kgA"] * 256 + g["len"] * 256) * 32 <= L.d * 32
+            assert (g["rt"] * 128 + 128) * 32 <= L.m * 32
+            assert (g["sl"] + 1) * b * 128 <= L.segs * b * 128
+            for kg in range(g["kgA"], g["kgA"] + g["len"]):
+                key = (g["l"], g["rt"], g["i"], kg)
+                assert key not in seen
+                seen.add(key)
+            gids.append(L.cg0 + g["cg"])
+            g = seg_next(tab, g, K.C)
+        assert sorted(set(gids)) == list(range(gids[0], gids[-1] + 1))
+        # the groups after the first, as the epilogue names them
+        first = seg_of(tab, s0, K.C)
+        l, cg = first["l"], first["cg"]
+        for gid in sorted(set(gids))[1:]:
+            l, cg = group_next(tab, l, cg)
+            assert tab[l].cg0 + cg == gid
+    assert len(seen) == sum(L.RT * L.n * L.KG for L in tab)
+
+
+def group_ws_bytes(shapes, b):
+    """Mirror of bs_group_workspace_bytes: all row-tile counters first (their places
+    depend on the shapes only), then each linear's partials, 256-byte aligned."""
+    C = 4 if b == 1 else 2
+    off = -(-sum(m // 128 for (m, d, n) in shapes) * 4 // 256) * 256
+    for (m, d, n) in shapes:
+        segs = (m // 128) * n * -(-(d // 256) // C)
+        off = -(-(off + segs * b * 128 * 4) // 256) * 256
+    return off
