@@ -51,7 +51,8 @@
  *    return BS_ERR_CUDA.  Device-side waits are bounded; a wait that runs out sets a
  *    sticky device error word that bs_get_device_error reports as BS_ERR_TIMEOUT.
  *  - Shapes: m % 128 == 0, d % 256 == 0, 128 <= m, d <= 65536, k == 16 on the GPU
- *    path (bs_block_bytes and bs_pack_record accept any k >= 1).
+ *    path (bs_block_bytes and bs_pack_record accept any k >= 1); "w/o AVD" stacks
+ *    (vanilla-SVD blocks, below) take any m, d up to 65536.
  *  - Alignment: device buffers 256-byte aligned; x, y, W_out and 1/s 16-byte
  *    aligned.  Violations return BS_ERR_ALIGNMENT.
  *  - Thread safety: a handle is not thread-safe; distinct handles are independent.
@@ -187,8 +188,9 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
  * The scratch is an 8 MiB array inside the library, held by every GPU that loads
  * it until exit.  Calls whose scratch (bs_workspace_bytes) would exceed 8 MiB return
  * BS_ERR_CAPACITY (e.g. 4096 x 4096 needs 0.5 MiB at n = 8, batch 1, and fits up to
- * n = 64 at batch 1, 32 at batch 2, 21 at batch 3, 16 at batch 4); batch > 4 returns
- * BS_ERR_INVALID_ARG; the current device must be the stack's (BS_ERR_INVALID_ARG).
+ * n = 64 at batch 1, 31 at batch 2, 21 at batch 3, 15 at batch 4); batch > 4 and
+ * "w/o AVD" stacks return BS_ERR_INVALID_ARG; the current device must be the stack's
+ * (BS_ERR_INVALID_ARG).
  * The first call on each device looks up the array's device address synchronously,
  * so make it before any stream capture.  All calls on a device, whatever their stack,
  * share the array: once bs_get_device_error has reported an error on any stack of a

@@ -113,3 +113,16 @@ def test_status_strings():
         s = R.bs_status_string(code)
         assert s and s != "unknown status"
     assert R.bs_status_string(99) == "unknown status"
+
+
+def test_no_alloc_capacity_figures_in_the_header():
+    """The header's worked example of the no-alloc scratch limit: 4096 x 4096 fits
+    n = 64 at batch 1 (the decode path's block limit), 31 at batch 2, 21 at batch 3 and
+    15 at batch 4 in 8 MiB, and one block more does not."""
+    import residual_block_decomp_b200 as R
+    cap = 8 << 20
+    for b, n_max in ((1, 64), (2, 31), (3, 21), (4, 15)):
+        assert R.bs_workspace_bytes(4096, 4096, 16, n_max, b) <= cap
+        if n_max < 64:
+            assert R.bs_workspace_bytes(4096, 4096, 16, n_max + 1, b) > cap
+    assert R.bs_workspace_bytes(4096, 4096, 16, 8, 1) == 256 + 8 * 65536   # 0.5 MiB
