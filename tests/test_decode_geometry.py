@@ -351,3 +351,31 @@ def group_ws_bytes(shapes, b):
         segs = (m // 128) * n * -(-(d // 256) // C)
         off = -(-(off + segs * b * 128 * 4) // 256) * 256
     return off
+
+
+@pytest.mark.parametrize("m,d,n", SHAPES)
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_bulk_copies_are_16_byte_units(m, d, n, b):
+    """Every 1-D bulk copy the decode kernel issues starts on a 16-byte boundary and
+    moves a multiple of 16 bytes (the rule of cp.async.bulk): sign stages, the first
+    group's V rows, 1/s and x rows, from a 256-byte aligned stack, 16-byte aligned 1/s
+    and x, into shared-memory regions at 1024-byte offsets."""
+    K, RT, KG, NCB, segs, grid = geometry(m, d, n, b)
+    block = m * d // 8 + 32 * (m + d)
+    assert block % 16 == 0 and (m * d // 8) % 16 == 0 and (m * d // 8 + 32 * m) % 16 == 0
+    for cg in range(n * NCB):
+        i, cgb = divmod(cg, NCB)
+        kgA = cgb * K.C
+        ln = min(K.C, KG - kgA)
+        gcols = ln * 256
+        col0 = kgA * 256
+        for rt in range(RT):
+            src = i * block + (rt * KG + kgA) * 4096
+            assert src % 16 == 0 and (ln * 4096) % 16 == 0
+        v_src = i * block + m * d // 8 + 32 * m + col0 * 32
+        assert v_src % 16 == 0 and (gcols * 32) % 16 == 0
+        assert (col0 * 4) % 16 == 0 and (gcols * 4) % 16 == 0            # 1/s
+        for lane in range(b):
+            assert (lane * d * 2 + col0 * 2) % 16 == 0 and (gcols * 2) % 16 == 0   # x row
+    # shared-memory destinations: sets, stages, control block, staging
+    assert (2 * K.SET) % 1024 == 0 and K.STAGE % 1024 == 0 and (2 * K.SET + K.NS * K.STAGE + 8192) % 1024 == 0
