@@ -300,6 +300,8 @@ def run_cuda(args, rank, world, local_rank):
         out["extras"] = extras(args, dev, stream, layers[0], ws, inv_s)
     for layer in layers:
         layer.close()
+    if args.extras and rank == 0:
+        out["extras"].update(extras_workloads(args, dev, stream, l2))
     return out
 
 
@@ -359,16 +361,238 @@ def extras(args, dev, stream, layer, ws, inv_s):
     return res
 
 
+def _graph_us(dev, stream, step, count, reps=3):
+    """Per-step µs of `count` steps replayed from one CUDA graph (best of `reps`)."""
+    import torch
+    for j in range(3):
+        step(j)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for j in range(count):
+            step(j)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1000.0 / count)
+    del g
+    return best
+
+
+def _stacks(m, d, n, count, gen, dev, plain=False, kp=None):
+    from residual_block_decomp_b200 import BitStackLinear
+    import residual_block_decomp_b200 as R
+    layers = []
+    for _ in range(count):
+        inv_s = wl.synthetic_inv_scale(d, gen)
+        if plain:
+            L = BitStackLinear(m, d, n, inv_s, k=kp, device=dev, plain=True)
+            for i in range(n):
+                U = wl.random_factors(m, kp, gen, 0.05 / np.sqrt(i + 1.0))
+                V = wl.random_factors(d, kp, gen, 0.05 / np.sqrt(i + 1.0))
+                L.add_record(np.concatenate([U.view(np.uint8).reshape(-1), V.view(np.uint8).reshape(-1)]))
+        else:
+            L = BitStackLinear(m, d, n, inv_s, device=dev)
+            for rec in make_records(m, d, K_HEAD, n, gen):
+                L.add_record(rec)
+        L.set_loaded(n)
+        layers.append(L)
+    return layers
+
+
+def extras_workloads(args, dev, stream, l2):
+    """The other workloads: the MLP linears (config 3), prefill shapes (config 4), the
+    whole-model token through a grouped launch (config 5), "w/o AVD" stacks, and the
+    headline call's latency with L2 flushed before every call."""
+    import torch
+    import residual_block_decomp_b200 as R
+    res = {}
+    gen = wl.generator(3, 0, "blocks")
+
+    # headline call, L2 flushed (a 4x-L2 buffer written) before every timed call
+    layers = _stacks(M_HEAD, D_HEAD, N_HEAD, 1, gen, dev)
+    x = torch.randn((1, D_HEAD), device=dev).half()
+    y = torch.empty((1, M_HEAD), device=dev, dtype=torch.float16)
+    ws = torch.zeros(R.bs_workspace_bytes(M_HEAD, D_HEAD, K_HEAD, N_HEAD, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(4 * l2 // 4, dtype=torch.float32, device=dev)
+    times = []
+    with torch.cuda.stream(stream):
+        for j in range(33):
+            flush.fill_(float(j))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layers[0].forward(x, N_HEAD, out=y, workspace=ws, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            if j >= 3:
+                times.append(e0.elapsed_time(e1) * 1000.0)
+    res["decode_l2_flushed_single_call_us"] = round(statistics.median(times), 3)
+    # eager end-to-end: pinned x in, one binding call, y out, no graph, per call
+    xh = torch.empty((1, D_HEAD), dtype=torch.float16, pin_memory=True)
+    yh = torch.empty((1, M_HEAD), dtype=torch.float16, pin_memory=True)
+    xh.copy_(x.cpu())
+    with torch.cuda.stream(stream):
+        for _ in range(20):
+            x.copy_(xh, non_blocking=True)
+            layers[0].forward(x, N_HEAD, out=y, workspace=ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        stream.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(500):
+            x.copy_(xh, non_blocking=True)
+            layers[0].forward(x, N_HEAD, out=y, workspace=ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        stream.synchronize()
+        res["decode_e2e_eager_us"] = round((time.perf_counter() - t0) * 1e6 / 500, 2)
+    for L in layers:
+        L.close()
+    del flush
+
+    # config 3: MLP linears, 12-block stacks, n per matrix drawn from 2..12, L2-rotated
+    for (m, d) in ((14336, 4096), (4096, 14336)):
+        count = max(2, int(np.ceil(3 * l2 / (12 * R.bs_block_bytes(m, d, K_HEAD)))) + 1)
+        layers = _stacks(m, d, 12, count, gen, dev)
+        ns = wl.n_loaded_draws(count, gen, 2, 12).tolist()
+        for b in (1, 4, 16):
+            xs = [torch.randn((b, d), device=dev).half() for _ in range(count)]
+            ys = [torch.empty((b, m), device=dev, dtype=torch.float16) for _ in range(count)]
+            wss = [L.workspace(12, b) for L in layers]
+
+            def step(j, layers=layers, xs=xs, ys=ys, wss=wss, ns=ns):
+                k = j % len(layers)
+                layers[k].forward(xs[k], ns[k], out=ys[k], workspace=wss[k], stream=stream)
+            us = _graph_us(dev, stream, step, 10 * count)
+            nbytes = np.mean([n * R.bs_block_bytes(m, d, K_HEAD) for n in ns])
+            res[f"mlp_{m}x{d}_b{b}_us"] = round(us, 2)
+            res[f"mlp_{m}x{d}_b{b}_hbm_frac"] = round(nbytes / (us * 1e-6) / 1e9 / peaks()[0], 4)
+        res[f"mlp_{m}x{d}_n_loaded"] = ns
+        for L in layers:
+            L.close()
+
+    # config 4: prefill, n = 8, M in {512, 2048, 4096}, bf16 tokens
+    for (m, d) in ((4096, 4096), (14336, 4096)):
+        layers = _stacks(m, d, 8, 1, gen, dev)
+        for M in (512, 2048, 4096):
+            xM = torch.randn((M, d), device=dev).bfloat16()
+            yM = torch.empty((M, m), device=dev, dtype=torch.bfloat16)
+            us = _graph_us(dev, stream, lambda j: layers[0].forward(xM, 8, out=yM, stream=stream), 5)
+            res[f"prefill_{m}x{d}_M{M}_us"] = round(us, 1)
+            res[f"prefill_{m}x{d}_M{M}_tensor_frac"] = round(2.0 * M * m * d / (us * 1e-6) / 1e12 / peaks()[1], 4)
+        layers[0].close()
+
+    # "w/o AVD": vanilla rank-k' blocks of the same bytes, 4096 x 4096, n = 8, batch 1
+    kp = R.bs_plain_rank(M_HEAD, D_HEAD, K_HEAD)
+    pbytes = N_HEAD * R.bs_plain_block_bytes(M_HEAD, D_HEAD, kp)
+    count = max(2, int(np.ceil(3 * l2 / pbytes)) + 1)
+    layers = _stacks(M_HEAD, D_HEAD, N_HEAD, count, gen, dev, plain=True, kp=kp)
+    x1 = torch.randn((1, D_HEAD), device=dev).half()
+    y1 = torch.empty((1, M_HEAD), device=dev, dtype=torch.float16)
+    wsp = layers[0].workspace(N_HEAD, 1)
+    us = _graph_us(dev, stream, lambda j: layers[j % count].forward(x1, N_HEAD, out=y1, workspace=wsp,
+                                                                    stream=stream), 10 * count)
+    res["plain_4096x4096_kp144_n8_b1_us"] = round(us, 3)
+    res["plain_4096x4096_kp144_n8_b1_hbm_frac"] = round(pbytes / (us * 1e-6) / 1e9 / peaks()[0], 4)
+    for L in layers:
+        L.close()
+    torch.cuda.synchronize(dev)
+
+    res.update(extras_model(dev, stream))
+    return res
+
+
+def extras_model(dev, stream, budgets_mib=(3000, 2000, 4500), tokens=20):
+    """Config 5: 224 Llama-3-8B-shaped linears with 16-block stacks; per-linear loaded
+    counts from the greedy fill of each budget over a Greedy global order (the
+    library's planner on seeded per-block scores); blocks dropped / appended between
+    budgets (timed); then one decode token through all linears, as one grouped launch
+    and as one launch per linear."""
+    import torch
+    import residual_block_decomp_b200 as R
+    from residual_block_decomp_b200 import BitStackLinear
+    mats = wl.llama3_8b_matrices()
+    shapes = [(m, d) for (_, _, m, d) in mats]
+    gen = wl.generator(5, 0, "blocks")
+    # one storage copy per (shape, level), shared by the stacks of that shape
+    pinned = {}
+    for (m, d) in sorted(set(shapes)):
+        recs = []
+        for rec in make_records(m, d, K_HEAD, 16, gen):
+            t = torch.empty(rec.size, dtype=torch.uint8, pin_memory=True)
+            t.copy_(torch.from_numpy(rec))
+            recs.append(t)
+        pinned[(m, d)] = recs
+    layers = []
+    for (m, d) in shapes:
+        L = BitStackLinear(m, d, 16, wl.synthetic_inv_scale(d, gen), device=dev)
+        for t in pinned[(m, d)]:
+            L.add_pinned_record(t)
+        layers.append(L)
+    sizes = np.array([R.bs_block_bytes(m, d, K_HEAD) for (m, d) in shapes], dtype=np.uint64)
+    # per-block scores: energy drop per byte from seeded geometric residual-norm decays
+    sgen = wl.generator(5, 0, "plan")
+    norms = np.cumprod(np.concatenate([np.ones((len(shapes), 1)), sgen.uniform(0.8, 0.99, (len(shapes), 16))], 1), 1)
+    scores = (norms[:, :-1] ** 2 - norms[:, 1:] ** 2) / sizes[:, None].astype(np.float64)
+    order_w, _ = R.bs_plan_order([16] * len(shapes), R.BS_ORDER_GREEDY, scores=scores)
+    xs = [torch.randn((1, d), device=dev).half() for (_, d) in shapes]
+    ys = [torch.empty((1, m), device=dev, dtype=torch.float16) for (m, _) in shapes]
+    handles = [L.handle for L in layers]
+    ws = None
+    out = {"model_linears": len(shapes)}
+    for mib in budgets_mib:
+        counts = R.bs_plan_budget(order_w, sizes, int(mib) * 2 ** 20).tolist()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        moved = sum(abs(c - L.n_blocks) * int(sz) for c, L, sz in zip(counts, layers, sizes))
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for L, c in zip(layers, counts):
+                L.set_loaded(c, stream=stream)
+            e1.record(stream)
+        e1.synchronize()
+        loaded = int(np.sum(np.array(counts, dtype=np.uint64) * sizes))
+        out[f"model_{mib}MiB_budget_change_ms"] = round(e0.elapsed_time(e1), 3)
+        out[f"model_{mib}MiB_bytes_moved"] = int(moved)
+        need = R.bs_group_workspace_bytes(handles, counts, 1)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        us_g = _graph_us(dev, stream, lambda j: R.bs_linear_group(handles, xs, counts, ys, ws, stream), tokens)
+        wss = [L.workspace(max(c, 1), 1) for L, c in zip(layers, counts)]
+
+        def token_singles(j):
+            for L, x, y, c, w in zip(layers, xs, ys, counts, wss):
+                L.forward(x, c, out=y, workspace=w, stream=stream)
+        us_s = _graph_us(dev, stream, token_singles, 3)
+        hbm = peaks()[0]
+        out[f"model_{mib}MiB_loaded_bytes"] = loaded
+        out[f"model_{mib}MiB_token_grouped_us"] = round(us_g, 1)
+        out[f"model_{mib}MiB_token_per_linear_launches_us"] = round(us_s, 1)
+        out[f"model_{mib}MiB_grouped_hbm_frac"] = round(loaded / (us_g * 1e-6) / 1e9 / hbm, 4)
+    assert layers[0].device_error() == 0
+    for L in layers:
+        L.close()
+    return out
+
+
 # -------------------------------------------------------------- oracle arm --------
 def run_oracle(args, budget_s):
-    """Times the oracle's factored float64 linear on the headline workload."""
+    """Times the oracle's two float64 forms of the linear on the headline workload, each
+    for about half of `budget_s`, with the BLAS pool pinned to the host's cores: the
+    factored form (the sign contraction per block) is the reported value, the explicit
+    form (rebuild the weight, then one product) is reported beside it."""
     from oracle import linear
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
-    except Exception:
-        threads = None
     cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=cores)
+    except Exception:
+        limiter = None
     m, d, k, n, b = args.m, args.d, K_HEAD, args.n, args.batch
     gen = wl.generator(2, 900, "blocks")
     negs, Us, Vs = [], [], []
@@ -379,17 +603,25 @@ def run_oracle(args, budget_s):
         Vs.append(V)
     inv_s = wl.synthetic_inv_scale(d, gen)
     x = wl.activations(b, d, gen).astype(np.float16)
-    calls = 0
-    t0 = time.perf_counter()
-    while True:
-        linear.linear_factored(x, negs, Us, Vs, inv_s, n, m)
-        calls += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    el = time.perf_counter() - t0
-    return {"value": el * 1e6 / calls, "unit": UNIT, "cores": threads or cores, "kind": "oracle",
-            "sample": f"{calls} call(s) of the float64 factored oracle on the full {m}x{d}, n={n}, k={k}, "
-                      f"batch {b} workload ({el:.1f} s); host has {cores} cores"}
+    timed = {}
+    for name, fn in (("factored", linear.linear_factored), ("explicit", linear.linear_explicit)):
+        calls = 0
+        t0 = time.perf_counter()
+        while True:
+            fn(x, negs, Us, Vs, inv_s, n, m)
+            calls += 1
+            if time.perf_counter() - t0 >= budget_s / 2:
+                break
+        timed[name] = (time.perf_counter() - t0, calls)
+    if limiter is not None:
+        limiter.restore_original_limits()
+    el, calls = timed["factored"]
+    ee, ce = timed["explicit"]
+    return {"value": el * 1e6 / calls, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "explicit_value": ee * 1e6 / ce,
+            "sample": f"{calls} call(s) of the float64 factored oracle ({el:.1f} s) and {ce} of the explicit "
+                      f"oracle ({ee:.1f} s) on the full {m}x{d}, n={n}, k={k}, batch {b} workload; BLAS threads "
+                      f"pinned to the {cores} host cores"}
 
 
 # ---------------------------------------------------------------------- main ------
@@ -411,7 +643,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    workload = f"decode {args.m}x{args.d} n={args.n} k={K_HEAD} batch={args.batch} fp16"
+    kind = "decode" if args.batch <= 4 else "prefill"
+    workload = f"{kind} {args.m}x{args.d} n={args.n} k={K_HEAD} batch={args.batch} fp16"
     config = {"workload": workload, "m": args.m, "d": args.d, "n_loaded": args.n, "k": K_HEAD,
               "batch": args.batch, "parallelism": f"replicas x{world}"}
 
