@@ -295,18 +295,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!failed) check(mbar_wait(&ctl->pfull[g], static_cast<uint32_t>((prounds >> 1) & 1), deadline, abort_flag));
         if (!failed) {
           tc_fence_after();
-          const int i1 = min(n, (r + 1) * kPRound);
-          for (int i = r * kPRound; i < i1; ++i) {
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_base + kPcol + 128u * g + (i - r * kPRound) * 32 + 16 * half, v);
-            const uint4 wq = *reinterpret_cast<const uint4*>(sbase + i * kTileBytes);
-            const uint32_t wd[4] = {wq.x, wq.y, wq.z, wq.w};
-            tc_wait_ld();
+          // the round's products and sign words all in flight before one wait
+          const int nbr = min(kPRound, n - r * kPRound);
+          uint32_t v[kPRound][16];
+          uint4 wq[kPRound];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              uint32_t x;
-              asm("mul.lo.u32 %0, %1, %2;" : "=r"(x) : "r"(wd[c >> 2]), "r"(mq[c & 3]));
-              acc[c] += __uint_as_float(v[c] ^ (x & 0x80000000u));
+          for (int ii = 0; ii < kPRound; ++ii) {
+            if (ii < nbr) {
+              tmem_ld16(tmem + lane_base + kPcol + 128u * g + ii * 32 + 16 * half, v[ii]);
+              wq[ii] = *reinterpret_cast<const uint4*>(sbase + (r * kPRound + ii) * kTileBytes);
+            }
+          }
+          tc_wait_ld();
+#pragma unroll
+          for (int ii = 0; ii < kPRound; ++ii) {
+            if (ii < nbr) {
+              const uint32_t wd[4] = {wq[ii].x, wq[ii].y, wq[ii].z, wq[ii].w};
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                uint32_t x;
+                asm("mul.lo.u32 %0, %1, %2;" : "=r"(x) : "r"(wd[c >> 2]), "r"(mq[c & 3]));
+                acc[c] += __uint_as_float(v[ii][c] ^ (x & 0x80000000u));
+              }
             }
           }
           tc_fence_before();
