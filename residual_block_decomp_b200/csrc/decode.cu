@@ -33,7 +33,7 @@
 //    which runs on the FMA pipe, then one AND per four columns; the device tile order)
 //    and stores them to one of its team's two slots in tensor memory; each warp then
 //    arrives on the slot's mbarrier.  No barrier inside a team.
-//  * MMA.  kNI issuer warps take the units in turn (warp-uniform, one elected lane
+//  * MMA.  NI issuer warps take the units in turn (warp-uniform, one elected lane
 //    issues): the unit's eight tcgen05.mma.kind::i8 (M = 128, N = 32 * batch, K = 32,
 //    s32 accumulate) into the segment's accumulator, then one commit that frees the slot
 //    and one that counts the unit into the segment's accumulator barrier.
@@ -60,7 +60,7 @@ namespace {
 
 constexpr int kMaxStages = 16;
 constexpr int kSlots = 2;              // tensor-memory A slots per team
-constexpr int kNI = 3;                 // issuer warps (20 warps in all at batch <= 2: 96 registers each)
+constexpr int kNI = 3;                 // the most issuer warps (20 warps in all at batch <= 2: 96 registers each)
 constexpr int kBarZ = 4;               // named barriers: 4 = all warps but the copy warp, 5 = epilogue
 constexpr int kBarEpi = 5;
 constexpr float kQMax = 32512.0f;      // |q| <= 127 * 256: q = 256 hi + lo with hi, lo in int8
@@ -81,8 +81,14 @@ struct Cfg {
   static constexpr int T = B <= 2 ? 3 : 2;          // teams of four warps
   static constexpr int NACC = B == 1 ? 4 : 2;       // segment accumulators in tensor memory
   static constexpr uint32_t ACOL0 = NACC * NB;      // first A-slot column (64 columns per slot)
-  static constexpr int WISS = 4 * T;                // issuer warps WISS .. WISS + kNI - 1
-  static constexpr int WEPI = 4 * T + kNI;          // epilogue warps WEPI .. WEPI + 3
+  // Issuer warps.  Issuer u % NI takes unit u, and unit u fills A slot
+  // ((u / T) % kSlots) of team u % T: NI divides T * kSlots, so every use of a slot goes
+  // to the same issuer, which therefore waits for the slot's uses one by one (a waiter
+  // that skipped a use could take an earlier phase of the same parity for the one it
+  // wants).
+  static constexpr int NI = B <= 2 ? 3 : 2;
+  static constexpr int WISS = 4 * T;                // issuer warps WISS .. WISS + NI - 1
+  static constexpr int WEPI = 4 * T + NI;           // epilogue warps WEPI .. WEPI + 3
   static constexpr int WCTL = WEPI + 4;             // copy thread, tensor-memory owner (last warp)
   static constexpr int THREADS = 32 * (WCTL + 1);
   static constexpr int ZTHREADS = THREADS - 32;     // warps that build the first sets
@@ -96,6 +102,7 @@ struct Cfg {
   static constexpr int NS = NS0 < kMaxStages ? NS0 : kMaxStages;
   static constexpr int SMEM = NS * STAGE + FIXED;
   static_assert(ACOL0 + T * kSlots * 64 <= 512, "tensor memory columns");
+  static_assert((T * kSlots) % NI == 0 && NI <= kNI, "each A slot has one issuer");
   static_assert(NS >= 4, "sign ring too small");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // each decode CTA allocates all 512 tensor-memory columns: two must never share an SM
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const __grid
       mbar_init(&ctl->vstage, 1);
       mbar_init(&ctl->xstage, 1);
       for (int z = 0; z < 2; ++z) mbar_init(&ctl->zready[z], 1);
-      for (int w = 0; w < kNI; ++w) mbar_init(&ctl->drain[w], 1);
+      for (int w = 0; w < K::NI; ++w) mbar_init(&ctl->drain[w], 1);
       ctl->abort = 0;
       ctl->nred = 0;
       ctl->count_ok = 0;
@@ -691,7 +698,7 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const __grid
       bool ok = true, any = false;
       Seg sg = sg0;
       while (j < nseg && ok) {
-        if (u % kNI == w) {
+        if (u % K::NI == w) {
           const int team = u % T, k = u / T, slot = k % kSlots, use = k / kSlots;
           const int a = j % NACC;
           // the slot's four quadrants are stored

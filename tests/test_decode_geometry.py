@@ -39,7 +39,7 @@ class Cfg:
         self.ZB = self.NB * 256
         self.SET = self.C * self.ZB
         self.T = 3 if b <= 2 else 2
-        self.NI = 3
+        self.NI = 3 if b <= 2 else 2
         self.NACC = 4 if b == 1 else 2
         self.ACOL0 = self.NACC * self.NB
         self.THREADS = 32 * (4 * self.T + self.NI + 5)
@@ -379,3 +379,16 @@ def test_bulk_copies_are_16_byte_units(m, d, n, b):
             assert (lane * d * 2 + col0 * 2) % 16 == 0 and (gcols * 2) % 16 == 0   # x row
     # shared-memory destinations: sets, stages, control block, staging
     assert (2 * K.SET) % 1024 == 0 and K.STAGE % 1024 == 0 and (2 * K.SET + K.NS * K.STAGE + 8192) % 1024 == 0
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_every_a_slot_has_one_issuer(b):
+    """Unit u goes to team u % T, A slot (u // T) % 2 of that team, and issuer u % NI.
+    The issuer waits on the slot's ready barrier by phase parity, so it must see every
+    use of the slot in turn: all uses of one slot go to one issuer."""
+    K = Cfg(b)
+    owner = {}
+    for u in range(10000):
+        slot = (u % K.T, (u // K.T) % 2)
+        assert owner.setdefault(slot, u % K.NI) == u % K.NI, (b, slot)
+    assert len(owner) == 2 * K.T and len(set(owner.values())) == K.NI
