@@ -504,6 +504,24 @@ def extras_workloads(args, dev, stream, l2):
         L.close()
     torch.cuda.synchronize(dev)
 
+    # the offline step on the GPU: decomposition of a 4096 x 4096 weight into 8 blocks
+    W = torch.randn((M_HEAD, D_HEAD), device=dev) * 0.02
+    sc = torch.rand(D_HEAD, device=dev) + 0.5
+    bb = R.bs_block_bytes(M_HEAD, D_HEAD, K_HEAD)
+    recs = torch.zeros(N_HEAD * bb, dtype=torch.uint8, device=dev)
+    norms = torch.zeros(N_HEAD + 1, dtype=torch.float64, device=dev)
+    dws = torch.empty(R.bs_decompose_workspace_bytes(M_HEAD, D_HEAD), dtype=torch.uint8, device=dev)
+    R.bs_decompose(W, sc, N_HEAD, recs, norms, dws, stream=stream)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        R.bs_decompose(W, sc, N_HEAD, recs, norms, dws, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    res["decompose_4096x4096_n8_ms"] = round(e0.elapsed_time(e1), 2)
+    del W, recs, dws
+
     res.update(extras_model(dev, stream))
     return res
 

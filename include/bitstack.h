@@ -210,6 +210,31 @@ bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_s
 /* out = S_block as int8 +-1, m x d row-major (block < n_blocks).  Asynchronous. */
 bs_status bs_unpack_signs(bs_stack_t stack, int block, int8_t* out, bs_stream_t stream);
 
+/* ------------------------------------------------------ GPU decomposition ----- */
+
+/* Workspace bytes bs_decompose needs for an m x d weight (0 for an unsupported shape):
+ * the fp32 residual (4 m d) plus sketches and small matrices, about 4 m d + 400 (m + d). */
+size_t bs_decompose_workspace_bytes(int m, int d, int k);
+
+/* Decomposes W into n_blocks BitStack records on the GPU (the offline step; review page
+ * "BitStack: Fine-Grained Size Control...", Figs. 3 and 5; OpenReview discussion, reply
+ * A3; README "Decomposition"): R_0 = W diag(s); for each block the sign bits of R
+ * (bit 1 where R < 0), the rank-k SVD of |R| with sqrt(sigma) folded into both fp16
+ * factors (each pair oriented so that the column sum of U is >= 0), and
+ * R <- R - S (.) (U V^T) with the stored fp16 factors.  The SVD is randomized subspace
+ * iteration with 32 columns, `power_iters` power iterations and a Gaussian sketch drawn
+ * from `seed` by a counter-based generator, so results differ from an exact SVD by the
+ * method's approximation, not by run.
+ * W: m x d fp32 row-major, s: d fp32 (the scale itself; the stack wants fp32 1/s), both
+ * device, 16-byte aligned.  records: device, >= n_blocks * bs_block_bytes(m, d, k),
+ * 256-aligned; record i at i * bs_block_bytes.  res_norms_sq: device, n_blocks + 1
+ * doubles, ||R_i||_F^2 for i = 0 .. n_blocks.  workspace: device, 256-aligned, at least
+ * bs_decompose_workspace_bytes.  Shapes as the GPU path (k == 16).  Asynchronous on
+ * `stream`; allocates nothing. */
+bs_status bs_decompose(int m, int d, int k, int n_blocks, const float* W, const float* s, unsigned long long seed,
+                       int power_iters, void* records, size_t records_bytes, double* res_norms_sq, void* workspace,
+                       size_t workspace_bytes, bs_stream_t stream);
+
 /* ------------------------------------------------- grouped decode (one launch) --- */
 
 /* A decode token through many linears in one launch.  The pages' use case is a whole

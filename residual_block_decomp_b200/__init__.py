@@ -12,7 +12,7 @@ _BINDING_NAMES = (
     "BS_BF16", "BS_ERR_ALIGNMENT", "BS_ERR_CAPACITY", "BS_ERR_CUDA", "BS_ERR_INVALID_ARG", "BS_ERR_NO_DEVICE",
     "BS_ERR_RANGE", "BS_ERR_TIMEOUT", "BS_ERR_UNSUPPORTED_SHAPE", "BS_F16", "BS_F32", "BS_OK", "BS_ORDER_AVERAGE",
     "BS_ORDER_GREEDY", "BS_ORDER_RANDOM", "EXPORTS",
-    "LIB_PATH", "BsError", "bs_append_block", "bs_block_bytes", "bs_debug_set_wait", "bs_drop_block",
+    "LIB_PATH", "BsError", "bs_append_block", "bs_block_bytes", "bs_decompose", "bs_decompose_workspace_bytes", "bs_debug_set_wait", "bs_drop_block",
     "bs_get_device_error", "bs_group_workspace_bytes", "bs_linear", "bs_linear_group", "bs_linear_no_alloc", "bs_pack_record", "bs_plain_block_bytes",
     "bs_plain_rank", "bs_plain_stack_create", "bs_plain_stack_device_bytes", "bs_plain_workspace_bytes",
     "bs_plan_budget", "bs_plan_order", "bs_reconstruct",

@@ -42,6 +42,7 @@ EXPORTS = (
     "bs_get_device_error", "bs_status_string", "bs_debug_set_wait", "bs_linear_no_alloc",
     "bs_plan_order", "bs_plan_budget", "bs_plain_rank", "bs_plain_block_bytes", "bs_plain_stack_device_bytes",
     "bs_plain_workspace_bytes", "bs_plain_stack_create", "bs_group_workspace_bytes", "bs_linear_group",
+    "bs_decompose_workspace_bytes", "bs_decompose",
 )
 
 
@@ -82,6 +83,8 @@ def _load():
         "bs_plain_stack_create": (I, [I, I, I, I, P, Z, P, P, ctypes.POINTER(P)]),
         "bs_group_workspace_bytes": (Z, [I, P, P, I]),
         "bs_linear_group": (I, [I, P, P, P, P, I, I, P, Z, P]),
+        "bs_decompose_workspace_bytes": (Z, [I, I, I]),
+        "bs_decompose": (I, [I, I, I, I, P, P, ctypes.c_ulonglong, I, P, Z, P, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -283,3 +286,19 @@ def bs_linear_group(handles, xs, n_loaded, ys, workspace, stream=None) -> None:
     st = lib.bs_linear_group(nl, _handles(handles), xp, yp, _ptr(counts), xs[0].shape[0], _dtype_code(xs[0]),
                              _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "bs_linear_group")
+
+
+def bs_decompose_workspace_bytes(m: int, d: int, k: int = 16) -> int:
+    return int(lib.bs_decompose_workspace_bytes(m, d, k))
+
+
+def bs_decompose(W, s, n_blocks: int, records, res_norms_sq, workspace, seed: int = 0, power_iters: int = 6,
+                 k: int = 16, stream=None) -> None:
+    """GPU decomposition of W (m x d fp32 CUDA tensor) with scale s (d fp32) into
+    n_blocks records (uint8 CUDA tensor) and the squared residual norms (n_blocks + 1
+    float64 CUDA tensor)."""
+    m, d = W.shape
+    st = lib.bs_decompose(m, d, k, n_blocks, _ptr(W), _ptr(s), int(seed), int(power_iters), _ptr(records),
+                          records.numel() * records.element_size(), _ptr(res_norms_sq), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bs_decompose")

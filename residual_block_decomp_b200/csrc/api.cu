@@ -446,6 +446,39 @@ bs_status bs_linear_group(int n_linears, const bs_stack_t* stacks, const void* c
   return cuda_status(launch_decode_group(p, batch, grid, stream));
 }
 
+size_t bs_decompose_workspace_bytes(int m, int d, int k) {
+  if (!gpu_shape_ok(m, d, k)) return 0;
+  return decompose_ws_layout(m, d).total;
+}
+
+bs_status bs_decompose(int m, int d, int k, int n_blocks, const float* W, const float* s, unsigned long long seed,
+                       int power_iters, void* records, size_t records_bytes, double* res_norms_sq, void* workspace,
+                       size_t workspace_bytes, bs_stream_t stream) {
+  if (W == nullptr || s == nullptr || records == nullptr || res_norms_sq == nullptr || workspace == nullptr ||
+      n_blocks <= 0 || n_blocks > 4096 || power_iters < 0 || power_iters > 64)
+    return BS_ERR_INVALID_ARG;
+  if (!gpu_shape_ok(m, d, k)) return BS_ERR_UNSUPPORTED_SHAPE;
+  const size_t bb = bs_block_bytes(m, d, k);
+  if (records_bytes < bb * static_cast<size_t>(n_blocks) || workspace_bytes < decompose_ws_layout(m, d).total)
+    return BS_ERR_CAPACITY;
+  if (!aligned(records, 256) || !aligned(workspace, 256) || !aligned(W, 16) || !aligned(s, 16) ||
+      !aligned(res_norms_sq, 8))
+    return BS_ERR_ALIGNMENT;
+  DecomposeArgs a{};
+  a.m = m;
+  a.d = d;
+  a.n = n_blocks;
+  a.power_iters = power_iters;
+  a.W = W;
+  a.s = s;
+  a.seed = seed;
+  a.records = static_cast<uint8_t*>(records);
+  a.block_bytes = bb;
+  a.res_norms = res_norms_sq;
+  a.workspace = workspace;
+  return cuda_status(run_decompose(a, stream));
+}
+
 bs_status bs_reconstruct(bs_stack_t stack, int n, void* W_out, bs_dtype dt, bs_stream_t stream) {
   if (stack == nullptr || W_out == nullptr) return BS_ERR_INVALID_ARG;
   if (dt != BS_F16 && dt != BS_BF16 && dt != BS_F32) return BS_ERR_INVALID_ARG;

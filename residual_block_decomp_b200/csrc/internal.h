@@ -117,6 +117,23 @@ cudaError_t launch_plain_reconstruct(const uint8_t* blocks, unsigned long long b
                                      const float* inv_s, int m, int d, int kp, int n, void* out, int dtype,
                                      cudaStream_t stream);
 
+// GPU decomposition (decompose.cu): workspace carve-up and arguments.
+struct DecomposeWs {
+  size_t R, Y, Y2, Z, Z2, Uf, Vf, small, total;
+};
+DecomposeWs decompose_ws_layout(int m, int d);
+struct DecomposeArgs {
+  int m, d, n, power_iters;
+  const float* W;            // m x d fp32, row-major
+  const float* s;            // d fp32: the activation-aware scale
+  unsigned long long seed;
+  uint8_t* records;          // n records of block_bytes
+  unsigned long long block_bytes;
+  double* res_norms;         // n + 1 squared Frobenius norms of the scaled residuals
+  void* workspace;
+};
+cudaError_t run_decompose(const DecomposeArgs& a, cudaStream_t stream);
+
 // Launchers (decode.cu, prefill.cu, aux_kernels.cu).  They return cudaSuccess or the
 // launch error.
 cudaError_t launch_decode(const DecodeParams& p, int batch, int grid, cudaStream_t stream);
