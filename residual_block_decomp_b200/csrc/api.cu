@@ -359,14 +359,31 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   p.n = n_loaded;
   p.M = batch;
   p.KG = d / kTileCols;
-  p.NT = batch >= 256 ? 256 : ((batch + 31) / 32) * 32;
+  // Token tile: 256 for long inputs, 128 up to 2047 tokens (more CTAs to fill the SMs),
+  // else the input rounded up to 32.  The CTAs of a row tile are clustered by up to 4
+  // along the tokens to share the rebuild of W_hat.
+  p.NT = batch >= 2048 ? 256 : (batch >= 128 ? 128 : ((batch + 31) / 32) * 32);
+  const int tiles = (batch + p.NT - 1) / p.NT;
+  p.CN = tiles >= 4 ? 4 : (tiles >= 2 ? 2 : 1);
   p.timeout_ns = stack->timeout_ns;
+  // Shared memory: fewer x stages first (never fewer than the cluster size: the kernel
+  // relies on XS >= CN), then one sign buffer, then smaller token tiles, then a smaller
+  // cluster.
   const size_t limit = 227 * 1024;
+  const int NT0 = p.NT;
   int xs = 4, sb = 2;
-  while (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit && xs > 2) --xs;
-  if (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit) sb = 1;
-  while (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit && p.NT > 32) p.NT /= 2;
-  if (prefill_smem_bytes(n_loaded, p.NT, xs, sb) > limit) return BS_ERR_CAPACITY;
+  for (;;) {
+    xs = 4;
+    sb = 2;
+    p.NT = NT0;
+    const int xs_min = p.CN > 2 ? p.CN : 2;
+    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && xs > xs_min) --xs;
+    if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit) sb = 1;
+    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && p.NT > 32) p.NT /= 2;
+    if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) <= limit) break;
+    if (p.CN == 1) return BS_ERR_CAPACITY;
+    p.CN /= 2;
+  }
   p.xstages = xs;
   p.sbufs = sb;
   CUtensorMap tm_x;

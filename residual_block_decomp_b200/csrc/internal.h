@@ -88,6 +88,7 @@ struct PrefillParams {
   uint32_t* err;
   int m, d, n, M, KG, NT;
   int xstages, sbufs;
+  int CN;                      // CTAs per cluster along the tokens sharing the W_hat rebuild (1, 2, 4)
   unsigned long long timeout_ns;
 };
 
@@ -142,7 +143,7 @@ size_t decode_smem_bytes(int batch);
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_u,
                            const CUtensorMap& tm_v, int bf16, cudaStream_t stream);
-size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs);
+size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs, int cn);
 
 // bs_linear_no_alloc keeps its scratch in one array per device, shared by every stack
 // on that device: an error reported on any stack marks the device's array for clearing

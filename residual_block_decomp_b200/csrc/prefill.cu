@@ -5,20 +5,30 @@
 // the OpenReview discussion of "BitStack: Any-Size Compression of Large Language
 // Models in Variable Memory Environments"; review page "BitStack: Fine-Grained Size
 // Control...", Figs. 3 and 5).  With many rows of x the dense contraction dominates,
-// so each CTA rebuilds tiles of W_hat on chip and never writes them to device memory:
+// so tiles of W_hat are rebuilt on chip and never written to device memory:
 //
-//   for each 32-column K-tile of its 128 output rows:
+//   for each 32-column K-tile of 128 output rows:
 //     P_i = U_i[rows] V_i[cols]^T          rank-16 tcgen05 MMA (fp16) -> TMEM, per block,
 //                                          four blocks per round, two rounds in flight
 //     W_t = (sum_i sign_i (.) P_i) / s     TMEM -> registers, sign applied by XOR
 //     W_t -> fp16/bf16 -> shared memory    the A operand of the GEMM
 //     y_tile += W_t x_tile^T               tcgen05 MMA, M = 128 rows, N = NT tokens
 //
+// The CTAs of one 128-row tile that take different token tiles form a cluster of CN
+// (1, 2 or 4) and share the rebuild: CTA rank r rebuilds the K-tiles kt = r (mod CN)
+// and writes each rebuilt tile into the W ring of every CTA of the cluster (distributed
+// shared memory), so a W tile is rebuilt once per cluster instead of once per CTA.
+// Ring slot kt mod WS (WS = 2 CN, so each rank owns two slots and can fill one while the
+// cluster still reads the other) is always filled by the same rank; a consumer's GEMM
+// hands the slot back to that rank with a multicast tcgen05.commit.
+//
 // Operands arrive by TMA (x tiles, U and V tiles; no multicast) and 1-D bulk copies
 // (sign tiles).  Warp roles: warps 0-7 rebuild (two warps per TMEM lane quadrant, each
 // taking half of a K-tile's columns; thread = row = TMEM lane) and write the epilogue,
-// warp 8 issues copies, warp 9 owns TMEM and issues MMAs.  All waits are bounded; a
-// wait that runs out sets the device error word and the CTA unwinds.
+// warp 8 copies x tiles, warp 10 copies the rebuild's U, V and sign tiles (so that
+// neither stream waits behind the other's flow control), warp 9 owns TMEM and issues
+// MMAs.  All mbarrier waits are
+// bounded; a wait that runs out sets the device error word and the CTA unwinds.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -28,17 +38,23 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kWarpLoad = 8, kWarpMma = 9;    // warps 0-7 rebuild (two per TMEM lane quadrant)
+constexpr int kWarpRbLoad = 10;               // U, V and sign tiles for the rebuild
 constexpr int kRb = 256;                      // rebuild threads
 constexpr int kKT = 32;              // K columns per tile
 constexpr int kPRound = 4;           // blocks per P round (one TMEM region of 128 columns)
 constexpr uint32_t kPcol = 256;      // TMEM columns of the two P regions (acc at 0..NT)
+constexpr int kVS = 2;               // V stages (the CTA's own K-tiles only)
+constexpr int kMaxWS = 8;            // W ring slots at most
+constexpr int kWTile = kTileRows * kKT * 2;   // bytes of one W tile
 
 struct Ctl {
   uint64_t ubar, accfull, drain;
   uint64_t pfull[2], pempty[2];      // P regions: products ready / read by the rebuild warps
-  uint64_t wfull[2], wempty[2];
+  uint64_t wfull[kMaxWS];            // W slot filled (armed with the tile's bytes, completed by its copy)
+  uint64_t wempty[kMaxWS];           // W slot read by every CTA of the cluster (one commit each)
+  uint64_t vfull[kVS], vempty[kVS];  // V stages of the own K-tiles
   uint32_t tmem_base;
   int abort;
 };
@@ -66,7 +82,7 @@ struct Layout {
   int u_off, s_off, x_off, v_off, w_off, ctl_off, total;
   int s_stride, x_stride, v_stride;
 };
-__host__ __device__ inline Layout prefill_layout(int n, int NT, int xstages, int sbufs) {
+__host__ __device__ inline Layout prefill_layout(int n, int NT, int xstages, int sbufs, int ws) {
   Layout L{};
   int off = 0;
   L.u_off = off;  off += n * 4096;                          // U tiles, 128 x 16 fp16 per block
@@ -75,8 +91,8 @@ __host__ __device__ inline Layout prefill_layout(int n, int NT, int xstages, int
   L.x_stride = NT * kKT * 2;
   L.x_off = off;  off += xstages * L.x_stride;              // x tiles, NT x 32
   L.v_stride = n * 1024;
-  L.v_off = off;  off += xstages * L.v_stride;              // V tiles, 32 x 16 per block
-  L.w_off = off;  off += 2 * kTileRows * kKT * 2;           // W_hat tiles, 128 x 32, double buffered
+  L.v_off = off;  off += kVS * L.v_stride;                  // V tiles of own K-tiles, 32 x 16 per block
+  L.w_off = off;  off += ws * kWTile;                       // W_hat tiles, 128 x 32, a ring of ws
   off = (off + 7) & ~7;
   L.ctl_off = off;
   off += static_cast<int>(sizeof(Ctl)) + 2 * xstages * 8 + 2 * sbufs * 8;
@@ -89,8 +105,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int n = p.n, NT = p.NT, XS = p.xstages, SB = p.sbufs;
-  const Layout L = prefill_layout(n, NT, XS, SB);
+  const int n = p.n, NT = p.NT, XS = p.xstages, SB = p.sbufs, CN = p.CN;
+  const int WS = CN > 1 ? 2 * CN : 2;               // W ring slots: two per rank of the cluster
+  const Layout L = prefill_layout(n, NT, XS, SB, WS);
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + L.ctl_off);
   uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + L.ctl_off + sizeof(Ctl));
   uint64_t* xempty = xfull + XS;
@@ -101,7 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rt = blockIdx.x;
   const int tok0 = blockIdx.y * NT;
+  const int rank = CN > 1 ? static_cast<int>(cluster_rank()) : 0;
   const int KT = p.d / kKT;
+  const int n_own = (KT - rank + CN - 1) / CN;      // own K-tiles rank, rank + CN, ...
   const int rounds = (n + kPRound - 1) / kPRound;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
   const uint32_t is_bf16 = std::is_same<DT, __nv_bfloat16>::value ? 1u : 0u;
@@ -114,9 +133,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
-    for (int w = 0; w < 2; ++w) {
-      mbar_init(&ctl->wfull[w], kRb);
-      mbar_init(&ctl->wempty[w], 1);
+    for (int w = 0; w < kMaxWS; ++w) {
+      mbar_init(&ctl->wfull[w], 1);        // armed by this CTA's MMA thread, filled by the producer's copy
+      mbar_init(&ctl->wempty[w], CN);      // one commit from every CTA of the cluster
+    }
+    for (int v = 0; v < kVS; ++v) {
+      mbar_init(&ctl->vfull[v], 1);
+      mbar_init(&ctl->vempty[v], 1);
     }
     for (int s = 0; s < XS; ++s) {
       mbar_init(&xfull[s], 1);
@@ -133,17 +156,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // every CTA's barriers are initialised before any CTA of the cluster arrives on them
+  if (CN > 1) cluster_sync();
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == kWarpLoad) {
-    // ----------------------------------------------------------------- loader -----
-    // The whole warp walks the K-tiles; lane 0 waits for free stages and sets the byte
-    // counts, then the lanes issue one copy each: issuing a copy costs the issuing
-    // thread a few hundred cycles, so spreading a K-tile's 2 n + 4 tensor copies (and a
-    // group's n sign copies) over the lanes keeps the loads ahead of the MMAs.
+    // ------------------------------------------------------------ x-tile loader -----
+    // x tiles for every K-tile (the GEMM's B operand), into a ring of XS stages; lane 0
+    // waits for a free stage, the lanes issue the tile's four copies in parallel.
+    const uint32_t FULL = 0xffffffffu;
+    if (lane == 0) prefetch_tmap(&tm_x);
+    bool ok = true;
+    int kt = 0;
+    for (; kt < KT && ok; ++kt) {
+      const int s = kt % XS, use = kt / XS;
+      if (lane == 0) {
+        if (use > 0) ok = mbar_wait(&xempty[s], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
+        if (ok) mbar_arrive_expect_tx(&xfull[s], static_cast<uint32_t>(NT) * kKT * 2u);
+      }
+      ok = __shfl_sync(FULL, ok, 0);
+      if (!ok) break;
+      uint8_t* xb = smem + L.x_off + s * L.x_stride;
+      if (lane < 4) tma_load_2d(xb + lane * NT * 16, &tm_x, kt * kKT + 8 * lane, tok0, &xfull[s]);
+    }
+    if (lane == 0) {
+      if (!ok) {
+        ctl->abort = 1;
+        atomicOr(p.err, kErrTimeout);
+      }
+      const uint64_t drain_by = globaltimer_ns() + 100000000ull;
+      for (int j = (kt > XS ? kt - XS : 0); j < kt; ++j)
+        mbar_wait(&xfull[j % XS], static_cast<uint32_t>((j / XS) & 1), drain_by, nullptr);
+    }
+  } else if (warp == kWarpRbLoad) {
+    // ---------------------------------------------------------- rebuild loader -----
+    // U tiles once; then, in K order, the sign group of every 8 K-tiles (all of the
+    // group's 8 K-tiles share its words; CN divides 8, so every group holds own K-tiles)
+    // and the V tiles of the CTA's own K-tiles, each as soon as its ring slot is free.
     const uint32_t FULL = 0xffffffffu;
     if (lane == 0) {
-      prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_u);
       prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(&ctl->ubar, static_cast<uint32_t>(n) * 4096u);
@@ -153,9 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(smem + L.u_off + (e >> 1) * 4096 + (e & 1) * 2048, &tm_u, 8 * (e & 1), rt * kTileRows, e >> 1,
                   &ctl->ubar);
     bool ok = true;
-    int kt = 0;
-    for (; kt < KT && ok; ++kt) {
-      if (kt % 8 == 0) {
+    int oi = 0, groups = 0;
+    for (; oi < n_own && ok; ++oi) {
+      const int kt = rank + oi * CN;
+      if (oi == 0 || (kt - CN) / 8 != kt / 8) {   // the first own K-tile of a sign group
         const int grp = kt / 8, sb = grp % SB, use = grp / SB;
         if (lane == 0) {
           if (use > 0) ok = mbar_wait(&sgempty[sb], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
@@ -168,20 +220,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (static_cast<size_t>(rt) * p.KG + grp) * kTileBytes;
           bulk_g2s(smem + L.s_off + sb * L.s_stride + i * kTileBytes, src, kTileBytes, &sgfull[sb]);
         }
+        ++groups;
       }
-      const int s = kt % XS, use = kt / XS;
+      const int vs = oi % kVS, vuse = oi / kVS;
       if (lane == 0) {
-        if (use > 0) ok = mbar_wait(&xempty[s], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
-        if (ok) mbar_arrive_expect_tx(&xfull[s], static_cast<uint32_t>(n) * 1024u + static_cast<uint32_t>(NT) * kKT * 2u);
+        if (vuse > 0) ok = mbar_wait(&ctl->vempty[vs], static_cast<uint32_t>((vuse - 1) & 1), deadline, abort_flag);
+        if (ok) mbar_arrive_expect_tx(&ctl->vfull[vs], static_cast<uint32_t>(n) * 1024u);
       }
       ok = __shfl_sync(FULL, ok, 0);
       if (!ok) break;
-      uint8_t* vb = smem + L.v_off + s * L.v_stride;
-      uint8_t* xb = smem + L.x_off + s * L.x_stride;
-      for (int e = lane; e < 2 * n + 4; e += 32) {
-        if (e < 2 * n) tma_load_3d(vb + (e >> 1) * 1024 + (e & 1) * 512, &tm_v, 8 * (e & 1), kt * kKT, e >> 1, &xfull[s]);
-        else tma_load_2d(xb + (e - 2 * n) * NT * 16, &tm_x, kt * kKT + 8 * (e - 2 * n), tok0, &xfull[s]);
-      }
+      uint8_t* vb = smem + L.v_off + vs * L.v_stride;
+      for (int e = lane; e < 2 * n; e += 32)
+        tma_load_3d(vb + (e >> 1) * 1024 + (e & 1) * 512, &tm_v, 8 * (e & 1), kt * kKT, e >> 1, &ctl->vfull[vs]);
     }
     if (lane == 0) {
       if (!ok) {
@@ -189,13 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(p.err, kErrTimeout);
       }
       // drain the copies issued last on every barrier
-      mbar_wait(&ctl->ubar, 0, globaltimer_ns() + 100000000ull, nullptr);
-      const int issued = kt;
-      for (int j = (issued > XS ? issued - XS : 0); j < issued; ++j)
-        mbar_wait(&xfull[j % XS], static_cast<uint32_t>((j / XS) & 1), globaltimer_ns() + 100000000ull, nullptr);
-      const int groups = (issued + 7) / 8;
+      const uint64_t drain_by = globaltimer_ns() + 100000000ull;
+      mbar_wait(&ctl->ubar, 0, drain_by, nullptr);
+      for (int j = (oi > kVS ? oi - kVS : 0); j < oi; ++j)
+        mbar_wait(&ctl->vfull[j % kVS], static_cast<uint32_t>((j / kVS) & 1), drain_by, nullptr);
       for (int g = (groups > SB ? groups - SB : 0); g < groups; ++g)
-        mbar_wait(&sgfull[g % SB], static_cast<uint32_t>((g / SB) & 1), globaltimer_ns() + 100000000ull, nullptr);
+        mbar_wait(&sgfull[g % SB], static_cast<uint32_t>((g / SB) & 1), drain_by, nullptr);
     }
   } else if (warp == kWarpMma) {
     // -------------------------------------------------------------- MMA issuer -----
@@ -204,17 +253,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_g = make_idesc(1u, is_bf16, is_bf16, 128u, static_cast<uint32_t>(NT));
       bool ok = mbar_wait(&ctl->ubar, 0, deadline, abort_flag);
       bool issued_any = false;
-      // P round pr = (K-tile, round) into TMEM region pr & 1: rank-16 products of up to
-      // kPRound blocks, once the K-tile's V rows have landed and the rebuild warps have
-      // read the region's previous round.
+      // P round pr = (own K-tile oi, round r) into TMEM region pr & 1: rank-16 products of
+      // up to kPRound blocks, once the tile's V rows have landed and the rebuild warps
+      // have read the region's previous round.  After a tile's last round the V stage
+      // is handed back (the commit fires when these MMAs are done).
       const uint32_t uaddr = smem_u32(smem + L.u_off);
       auto issue_p = [&](int pr) -> bool {
-        const int ktp = pr / rounds, r = pr - ktp * rounds, s = ktp % XS, g = pr & 1;
-        if (!mbar_wait(&xfull[s], static_cast<uint32_t>((ktp / XS) & 1), deadline, abort_flag)) return false;
+        const int oip = pr / rounds, r = pr - oip * rounds, g = pr & 1, vs = oip % kVS;
+        if (r == 0 && !mbar_wait(&ctl->vfull[vs], static_cast<uint32_t>((oip / kVS) & 1), deadline, abort_flag))
+          return false;
         if (pr >= 2 && !mbar_wait(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1), deadline, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t vaddr = smem_u32(smem + L.v_off + s * L.v_stride);
+        const uint32_t vaddr = smem_u32(smem + L.v_off + vs * L.v_stride);
         const int i1 = min(n, (r + 1) * kPRound);
         for (int i = r * kPRound; i < i1; ++i) {
           const uint64_t adesc = smem_desc_noswizzle(uaddr + i * 4096, 2048, 128);
@@ -223,32 +274,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         issued_any = true;
         tc_commit(&ctl->pfull[g]);
+        if (r == rounds - 1) tc_commit(&ctl->vempty[vs]);
         return true;
       };
-      // One thread, a fixed order whose every wait is for an event the other warps produce
-      // without waiting on a later step of this thread: the P rounds of K-tile kg + 1
-      // (their regions free up as the rebuild warps finish the rounds of kg), then the
-      // GEMM of K-tile kg once its W_hat tile is in shared memory.  Blocking waits keep
-      // this thread off the issue slots the rebuild warps need.
-      const int PR = KT * rounds;
+      // One thread, a fixed order in which every wait is for an event that depends only
+      // on steps of smaller K-tile index (of this CTA or of the cluster): the GEMM of
+      // K-tile kg once its W_hat tile is in this CTA's ring (the slot goes back to its
+      // producer, rank kg mod CN, when the GEMM is done), then the P rounds of the CTA's
+      // own K-tiles up to kg + CN.  Those tiles' V rows can land by then: the loader
+      // reaches K-tile kt after the GEMM of kt - XS, and XS >= CN.
+      const int PR = n_own * rounds;
       int pr = 0;
-      for (; pr < rounds && ok; ++pr) ok = issue_p(pr);
+      // every W slot expects one tile's bytes for its first use
+      for (int w = 0; w < WS && w < KT; ++w) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);
+      for (; pr < min(PR, rounds) && ok; ++pr) ok = issue_p(pr);   // the first own K-tile
       for (int kg = 0; kg < KT && ok; ++kg) {
-        for (; pr < min(PR, (kg + 2) * rounds) && ok; ++pr) ok = issue_p(pr);
-        const int w = kg & 1;
-        if (ok) ok = mbar_wait(&ctl->wfull[w], static_cast<uint32_t>((kg >> 1) & 1), deadline, abort_flag);
+        const int w = kg % WS;
+        if (ok) ok = mbar_wait_cluster(&ctl->wfull[w], static_cast<uint32_t>((kg / WS) & 1), deadline, abort_flag);
         if (!ok) break;
+        if (kg + WS < KT) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);   // the slot's next use
         tc_fence_after();
         const int s = kg % XS;
-        const uint32_t waddr = smem_u32(smem + L.w_off + w * kTileRows * kKT * 2);
+        if (ok) ok = mbar_wait(&xfull[s], static_cast<uint32_t>((kg / XS) & 1), deadline, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t waddr = smem_u32(smem + L.w_off + w * kWTile);
         const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
         for (int kk = 0; kk < 2; ++kk) {
           const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
           const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
           mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&ctl->wempty[w]);
-        tc_commit(&xempty[s]);   // the stage's V rows (read by this K-tile's P rounds) and x tile
+        issued_any = true;
+        tc_commit(&xempty[s]);
+        if (kg + WS < KT) {
+          if (CN > 1) tc_commit_multicast(&ctl->wempty[w], static_cast<uint16_t>(1u << (kg % CN)));
+          else tc_commit(&ctl->wempty[w]);
+        }
+        const int own_upto = (kg + CN - rank) / CN + 1;   // own K-tiles <= kg + CN
+        for (; pr < min(PR, own_upto * rounds) && ok; ++pr) ok = issue_p(pr);
       }
       if (ok) {
         tc_commit(&ctl->accfull);
@@ -271,10 +335,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) failed = true;
     };
     int prounds = 0;
-    for (int kt = 0; kt < KT; ++kt) {
+    // the CTA's own K-tiles kt = rank, rank + CN, ...; each is written into ring slot
+    // kt mod WS of every CTA of the cluster
+    for (int oi = 0; oi < n_own; ++oi) {
+      const int kt = rank + oi * CN;
       const int grp = kt / 8, t = kt % 8, sb = grp % SB;
-      const int w = kt & 1;
-      if (t == 0 && !failed) check(mbar_wait(&sgfull[sb], static_cast<uint32_t>((grp / SB) & 1), deadline, abort_flag));
+      const int w = kt % WS;
+      const bool first_in_group = oi == 0 || (kt - CN) / 8 != grp;
+      const bool last_in_group = oi + 1 == n_own || (kt + CN) / 8 != grp;
+      if (first_in_group && !failed)
+        check(mbar_wait(&sgfull[sb], static_cast<uint32_t>((grp / SB) & 1), deadline, abort_flag));
       // column c of the K-tile is bit 8 (c % 4) + t of word c / 4 of the row; a multiply by
       // 2^(31 - 8 (c % 4) - t) moves it to bit 31 on the FMA pipe, leaving one AND-XOR
       // (the integer pipe) and one add per element and block
@@ -324,21 +394,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++prounds;
       }
-      if (!failed && t == 7) mbar_arrive(&sgempty[sb]);
+      if (!failed && last_in_group) mbar_arrive(&sgempty[sb]);
       uint32_t packed[8];
 #pragma unroll
       for (int c = 0; c < 16; c += 2) packed[c / 2] = pack2<DT>(acc[c] * isv[c], acc[c + 1] * isv[c + 1]);
-      if (kt >= 2 && !failed) check(mbar_wait(&ctl->wempty[w], static_cast<uint32_t>(((kt >> 1) - 1) & 1), deadline, abort_flag));
+      // the slot is free in every CTA of the cluster once all their GEMMs of the tile
+      // WS earlier (also this rank's) are done
+      if (kt >= WS && !failed)
+        check(mbar_wait_cluster(&ctl->wempty[w], static_cast<uint32_t>(((kt / WS) - 1) & 1), deadline, abort_flag));
       if (!failed) {
-        uint8_t* wb = smem + L.w_off + w * kTileRows * kKT * 2;
 #pragma unroll
         for (int k2 = 0; k2 < 2; ++k2) {
           const int kc = 2 * half + k2;   // 8-column K chunk of the tile
-          *reinterpret_cast<uint4*>(wb + kc * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
+          *reinterpret_cast<uint4*>(smem + L.w_off + w * kWTile + kc * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
               make_uint4(packed[4 * k2], packed[4 * k2 + 1], packed[4 * k2 + 2], packed[4 * k2 + 3]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&ctl->wfull[w]);
+        fence_proxy_async_smem();   // read next by the copy engine and the tensor cores
+      }
+      // all rebuild warps pass here whatever failed (one decision for all of them); then
+      // one thread sends the tile from this CTA's slot to the same slot of every other CTA
+      // of the cluster, each copy completing the receiver's barrier, and completes its own
+      if (bar_any(1, kRb, failed)) {
+        failed = true;
+      } else if (threadIdx.x == 0) {
+        const uint8_t* src = smem + L.w_off + w * kWTile;
+        for (int c = 0; c < CN; ++c) {
+          if (c == rank) continue;
+          bulk_s2cluster(mapa_shared(smem_u32(src), static_cast<uint32_t>(c)), src, kWTile,
+                         mapa_shared(smem_u32(&ctl->wfull[w]), static_cast<uint32_t>(c)));
+        }
+        mbar_complete_tx(&ctl->wfull[w], kWTile);
       }
     }
     // epilogue: accumulator row `tid` holds NT token outputs; the two halves take
@@ -367,6 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
+  // no CTA leaves while another CTA of the cluster may still write its ring or arrive on
+  // its barriers
+  if (CN > 1) cluster_sync();
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -375,14 +463,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs) {
-  return static_cast<size_t>(prefill_layout(n, NT, xstages, sbufs).total) + 64;
+size_t prefill_smem_bytes(int n, int NT, int xstages, int sbufs, int cn) {
+  return static_cast<size_t>(prefill_layout(n, NT, xstages, sbufs, cn > 1 ? 2 * cn : 2).total) + 64;
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_u,
                            const CUtensorMap& tm_v, int bf16, cudaStream_t stream) {
-  const size_t smem = prefill_smem_bytes(p.n, p.NT, p.xstages, p.sbufs);
-  dim3 grid(p.m / kTileRows, (p.M + p.NT - 1) / p.NT);
+  const size_t smem = prefill_smem_bytes(p.n, p.NT, p.xstages, p.sbufs, p.CN);
+  // token tiles padded to a whole number of clusters (the extra CTAs rebuild their share
+  // and store nothing)
+  const int tiles = (p.M + p.NT - 1) / p.NT;
+  const int gy = (tiles + p.CN - 1) / p.CN * p.CN;
   // the attribute is per device and kernel: set it once for each (device, dtype), outside
   // any stream capture (the first call on a device must not be captured)
   static bool configured[64][2] = {};
@@ -398,12 +489,20 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, cons
     if (e != cudaSuccess) return e;
     configured[dev][bf16 ? 1 : 0] = true;
   }
-  if (bf16) {
-    prefill_kernel<__nv_bfloat16><<<grid, kThreads, smem, stream>>>(p, tm_x, tm_u, tm_v);
-  } else {
-    prefill_kernel<__half><<<grid, kThreads, smem, stream>>>(p, tm_x, tm_u, tm_v);
-  }
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(p.CN);
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.stream = stream;
+  cfg.gridDim = dim3(static_cast<unsigned>(p.m / kTileRows), static_cast<unsigned>(gy));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  if (bf16) return cudaLaunchKernelEx(&cfg, prefill_kernel<__nv_bfloat16>, p, tm_x, tm_u, tm_v);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<__half>, p, tm_x, tm_u, tm_v);
 }
 
 }  // namespace bs

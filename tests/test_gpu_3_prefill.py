@@ -16,6 +16,8 @@ pytestmark = pytest.mark.gpu
     (384, 1024, 9, 100, "bf16"),    # two P rounds (n > 8)
     (512, 768, 12, 300, "f16"),     # two token tiles, the second ragged
     (1024, 2048, 8, 16, "f16"),     # a decode batch of 16 through the prefill path
+    (640, 2560, 5, 600, "bf16"),    # five token tiles: clusters of 4 sharing the rebuild, the last padded
+    (256, 1024, 16, 2100, "f16"),   # 256-token tiles in clusters of 4, 16 blocks
 ])
 def test_prefill_shapes(m, d, n, M, dtype):
     st = cases.synthetic_stack(94, m, d, n, matrix=m + n)
