@@ -12,6 +12,8 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+constexpr cuuint32_t kKTile = 32;   // K columns per prefill K-tile
+
 bool gpu_shape_ok(int m, int d, int k) {
   return k == kK && m >= kTileRows && d >= kTileCols && m <= 65536 && d <= 65536 && m % kTileRows == 0 &&
          d % kTileCols == 0;
@@ -44,13 +46,13 @@ EncodeTiledFn encode_fn() {
 // Tensor map over a tensor of fp16/bf16 elements; dims / strides innermost first,
 // strides in bytes for dims 1.., box in elements.  No swizzle, no interleave.
 bool encode(CUtensorMap* map, bool bf16, int rank, void* base, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
+            const cuuint32_t* box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r =
       fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<cuuint32_t>(rank),
-         base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -389,8 +391,11 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   CUtensorMap tm_x;
   const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(batch)};
   const cuuint64_t xstr[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t xbox[2] = {8, static_cast<cuuint32_t>(p.NT)};
-  if (!encode(&tm_x, dt == BS_BF16, 2, const_cast<void*>(x), xdims, xstr, xbox)) return BS_ERR_CUDA;
+  // one 32-column K-tile of NT tokens per copy: rows of 64 bytes in the 64-byte swizzle
+  // layout the GEMM reads x in
+  const cuuint32_t xbox[2] = {kKTile, static_cast<cuuint32_t>(p.NT)};
+  if (!encode(&tm_x, dt == BS_BF16, 2, const_cast<void*>(x), xdims, xstr, xbox, CU_TENSOR_MAP_SWIZZLE_64B))
+    return BS_ERR_CUDA;
   return cuda_status(launch_prefill(p, tm_x, stack->tm_u, stack->tm_v, dt == BS_BF16 ? 1 : 0, stream));
 }
 

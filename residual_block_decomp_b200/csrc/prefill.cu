@@ -22,8 +22,8 @@
 // cluster still reads the other) is always filled by the same rank; a consumer's GEMM
 // hands the slot back to that rank with a multicast tcgen05.commit.
 //
-// Operands arrive by TMA (x tiles, U and V tiles; no multicast) and 1-D bulk copies
-// (sign tiles).  Warp roles: warps 0-7 rebuild (two warps per TMEM lane quadrant, each
+// Operands arrive by TMA (x tiles in the 64-byte swizzle layout, U and V tiles; no
+// multicast) and 1-D bulk copies (sign tiles).  Warp roles: warps 0-7 rebuild (two warps per TMEM lane quadrant, each
 // taking half of a K-tile's columns; thread = row = TMEM lane) and write the epilogue,
 // warp 8 copies x tiles, warp 10 copies the rebuild's U, V and sign tiles (so that
 // neither stream waits behind the other's flow control), warp 9 owns TMEM and issues
@@ -176,8 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = __shfl_sync(FULL, ok, 0);
       if (!ok) break;
-      uint8_t* xb = smem + L.x_off + s * L.x_stride;
-      if (lane < 4) tma_load_2d(xb + lane * NT * 16, &tm_x, kt * kKT + 8 * lane, tok0, &xfull[s]);
+      if (lane == 0) tma_load_2d(smem + L.x_off + s * L.x_stride, &tm_x, kt * kKT, tok0, &xfull[s]);
     }
     if (lane == 0) {
       if (!ok) {
@@ -302,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
         for (int kk = 0; kk < 2; ++kk) {
           const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
-          const uint64_t bdesc = smem_desc_noswizzle(xaddr + kk * 2 * NT * 16, NT * 16, 128);
+          // x: NT rows of 64 bytes (64-byte swizzle), K-step kk = bytes 32 kk of each row
+          const uint64_t bdesc = smem_desc_sw64(xaddr + kk * 32, 8 * 64);
           mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
         }
         issued_any = true;

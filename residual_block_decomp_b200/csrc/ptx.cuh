@@ -290,6 +290,19 @@ __device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t smem_addr, uint
   desc |= static_cast<uint64_t>(1) << 46;
   return desc;  // base offset 0, lbo mode 0, layout type 0 (no swizzle)
 }
+// K-major operand in the 64-byte swizzle layout (rows of 64 bytes, 16-byte chunks
+// permuted by the row index, as a TMA load with 64-byte swizzle writes them), 8-row groups
+// `sbo` bytes apart; the tile base 512-byte aligned.  A K-step inside the 64-byte row is
+// selected by advancing the start address.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t smem_addr, uint32_t sbo) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  desc |= static_cast<uint64_t>(1) << 16;                       // leading offset: unused here
+  desc |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  desc |= static_cast<uint64_t>(1) << 46;
+  desc |= static_cast<uint64_t>(4) << 61;                       // layout type: 64-byte swizzle
+  return desc;
+}
 
 // Instruction descriptors (kind::f16 / kind::i8), dense, both operands K-major.
 // c_format: 0 f16, 1 f32, 2 s32.  a/b format: kind::f16 -> 0 f16, 1 bf16;
