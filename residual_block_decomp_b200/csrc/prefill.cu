@@ -26,8 +26,9 @@
 // multicast) and 1-D bulk copies (sign tiles).  Warp roles: warps 0-7 rebuild (two warps per TMEM lane quadrant, each
 // taking half of a K-tile's columns; thread = row = TMEM lane) and write the epilogue,
 // warp 8 copies x tiles, warp 10 copies the rebuild's U, V and sign tiles (so that
-// neither stream waits behind the other's flow control), warp 9 owns TMEM and issues
-// MMAs.  All mbarrier waits are
+// neither stream waits behind the other's flow control), warp 9 owns TMEM and issues the
+// GEMM, warp 11 issues the rank-16 products (two MMA streams that never wait on each
+// other).  All mbarrier waits are
 // bounded; a wait that runs out sets the device error word and the CTA unwinds.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -38,9 +39,10 @@
 namespace bs {
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kWarpLoad = 8, kWarpMma = 9;    // warps 0-7 rebuild (two per TMEM lane quadrant)
 constexpr int kWarpRbLoad = 10;               // U, V and sign tiles for the rebuild
+constexpr int kWarpP = 11;                    // issues the rank-16 products of the rebuild
 constexpr int kRb = 256;                      // rebuild threads
 constexpr int kKT = 32;              // K columns per tile
 constexpr int kPRound = 4;           // blocks per P round (one TMEM region of 128 columns)
@@ -50,7 +52,7 @@ constexpr int kMaxWS = 8;            // W ring slots at most
 constexpr int kWTile = kTileRows * kKT * 2;   // bytes of one W tile
 
 struct Ctl {
-  uint64_t ubar, accfull, drain;
+  uint64_t ubar, accfull, drain, drain_p;
   uint64_t pfull[2], pempty[2];      // P regions: products ready / read by the rebuild warps
   uint64_t wfull[kMaxWS];            // W slot filled (armed with the tile's bytes, completed by its copy)
   uint64_t wempty[kMaxWS];           // W slot read by every CTA of the cluster (one commit each)
@@ -133,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->drain_p, 1);
     for (int w = 0; w < kMaxWS; ++w) {
       mbar_init(&ctl->wfull[w], 1);        // armed by this CTA's MMA thread, filled by the producer's copy
       mbar_init(&ctl->wempty[w], CN);      // one commit from every CTA of the cluster
@@ -245,24 +248,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = (groups > SB ? groups - SB : 0); g < groups; ++g)
         mbar_wait(&sgfull[g % SB], static_cast<uint32_t>((g / SB) & 1), drain_by, nullptr);
     }
-  } else if (warp == kWarpMma) {
-    // -------------------------------------------------------------- MMA issuer -----
+  } else if (warp == kWarpP) {
+    // ------------------------------------------------------- product issuer -----
+    // P round pr = (own K-tile oi, round r) into TMEM region pr & 1: rank-16 products of
+    // up to kPRound blocks, once the tile's V rows have landed and the rebuild warps have
+    // read the region's previous round.  After a tile's last round its V stage is handed
+    // back (the commit fires when these MMAs are done).  Runs ahead of the GEMM as far as
+    // the V stages and the two regions allow.
     if (lane == 0) {
       const uint32_t idesc_p = make_idesc(1u, 0u, 0u, 128u, 32u);                 // f32 <- f16 x f16
-      const uint32_t idesc_g = make_idesc(1u, is_bf16, is_bf16, 128u, static_cast<uint32_t>(NT));
       bool ok = mbar_wait(&ctl->ubar, 0, deadline, abort_flag);
       bool issued_any = false;
-      // P round pr = (own K-tile oi, round r) into TMEM region pr & 1: rank-16 products of
-      // up to kPRound blocks, once the tile's V rows have landed and the rebuild warps
-      // have read the region's previous round.  After a tile's last round the V stage
-      // is handed back (the commit fires when these MMAs are done).
       const uint32_t uaddr = smem_u32(smem + L.u_off);
-      auto issue_p = [&](int pr) -> bool {
+      const int PR = n_own * rounds;
+      for (int pr = 0; pr < PR && ok; ++pr) {
         const int oip = pr / rounds, r = pr - oip * rounds, g = pr & 1, vs = oip % kVS;
-        if (r == 0 && !mbar_wait(&ctl->vfull[vs], static_cast<uint32_t>((oip / kVS) & 1), deadline, abort_flag))
-          return false;
-        if (pr >= 2 && !mbar_wait(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1), deadline, abort_flag))
-          return false;
+        if (r == 0) ok = mbar_wait(&ctl->vfull[vs], static_cast<uint32_t>((oip / kVS) & 1), deadline, abort_flag);
+        if (ok && pr >= 2)
+          ok = mbar_wait(&ctl->pempty[g], static_cast<uint32_t>(((pr >> 1) - 1) & 1), deadline, abort_flag);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t vaddr = smem_u32(smem + L.v_off + vs * L.v_stride);
         const int i1 = min(n, (r + 1) * kPRound);
@@ -274,27 +278,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued_any = true;
         tc_commit(&ctl->pfull[g]);
         if (r == rounds - 1) tc_commit(&ctl->vempty[vs]);
-        return true;
-      };
-      // One thread, a fixed order in which every wait is for an event that depends only
-      // on steps of smaller K-tile index (of this CTA or of the cluster): the GEMM of
-      // K-tile kg once its W_hat tile is in this CTA's ring (the slot goes back to its
-      // producer, rank kg mod CN, when the GEMM is done), then the P rounds of the CTA's
-      // own K-tiles up to kg + CN.  Those tiles' V rows can land by then: the loader
-      // reaches K-tile kt after the GEMM of kt - XS, and XS >= CN.
-      const int PR = n_own * rounds;
-      int pr = 0;
+      }
+      if (!ok) {
+        ctl->abort = 1;
+        atomicOr(p.err, kErrTimeout);
+      }
+      if (issued_any) {   // no product may still write tensor memory at exit
+        tc_commit(&ctl->drain_p);
+        mbar_wait(&ctl->drain_p, 0, globaltimer_ns() + 100000000ull, nullptr);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ----------------------------------------------------------- GEMM issuer -----
+    // The GEMM of K-tile kg once its W_hat tile is in this CTA's ring and its x tile has
+    // landed; the slot goes back to its producer (rank kg mod CN) when the GEMM is done.
+    // Every wait is for an event that depends only on smaller K-tiles.
+    if (lane == 0) {
+      const uint32_t idesc_g = make_idesc(1u, is_bf16, is_bf16, 128u, static_cast<uint32_t>(NT));
+      bool ok = true;
+      bool issued_any = false;
       // every W slot expects one tile's bytes for its first use
       for (int w = 0; w < WS && w < KT; ++w) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);
-      for (; pr < min(PR, rounds) && ok; ++pr) ok = issue_p(pr);   // the first own K-tile
       for (int kg = 0; kg < KT && ok; ++kg) {
         const int w = kg % WS;
-        if (ok) ok = mbar_wait_cluster(&ctl->wfull[w], static_cast<uint32_t>((kg / WS) & 1), deadline, abort_flag);
+        ok = mbar_wait_cluster(&ctl->wfull[w], static_cast<uint32_t>((kg / WS) & 1), deadline, abort_flag);
         if (!ok) break;
         if (kg + WS < KT) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);   // the slot's next use
-        tc_fence_after();
         const int s = kg % XS;
-        if (ok) ok = mbar_wait(&xfull[s], static_cast<uint32_t>((kg / XS) & 1), deadline, abort_flag);
+        ok = mbar_wait(&xfull[s], static_cast<uint32_t>((kg / XS) & 1), deadline, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t waddr = smem_u32(smem + L.w_off + w * kWTile);
@@ -311,8 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (CN > 1) tc_commit_multicast(&ctl->wempty[w], static_cast<uint16_t>(1u << (kg % CN)));
           else tc_commit(&ctl->wempty[w]);
         }
-        const int own_upto = (kg + CN - rank) / CN + 1;   // own K-tiles <= kg + CN
-        for (; pr < min(PR, own_upto * rounds) && ok; ++pr) ok = issue_p(pr);
       }
       if (ok) {
         tc_commit(&ctl->accfull);
