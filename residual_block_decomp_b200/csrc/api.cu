@@ -368,9 +368,8 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   const int tiles = (batch + p.NT - 1) / p.NT;
   p.CN = tiles >= 4 ? 4 : (tiles >= 2 ? 2 : 1);
   p.timeout_ns = stack->timeout_ns;
-  // Shared memory: fewer x stages first (never fewer than the cluster size: the kernel
-  // relies on XS >= CN), then one sign buffer, then smaller token tiles, then a smaller
-  // cluster.
+  // Shared memory: fewer x stages first (down to two), then one sign buffer, then smaller
+  // token tiles, then a smaller cluster.
   const size_t limit = 227 * 1024;
   const int NT0 = p.NT;
   int xs = 4, sb = 2;
@@ -378,8 +377,7 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
     xs = 4;
     sb = 2;
     p.NT = NT0;
-    const int xs_min = p.CN > 2 ? p.CN : 2;
-    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && xs > xs_min) --xs;
+    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && xs > 2) --xs;
     if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit) sb = 1;
     while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && p.NT > 32) p.NT /= 2;
     if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) <= limit) break;
