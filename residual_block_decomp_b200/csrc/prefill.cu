@@ -299,29 +299,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued_any = false;
       // every W slot expects one tile's bytes for its first use
       for (int w = 0; w < WS && w < KT; ++w) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);
+      // ring positions kept as counters (no divisions in the loop): W slot w of use wu,
+      // x stage s of use su, producer rank pk = kg mod CN
+      const uint64_t adesc0 = smem_desc_noswizzle(smem_u32(smem + L.w_off), 2048, 128);
+      const uint64_t bdesc0 = smem_desc_sw64(smem_u32(smem + L.x_off), 8 * 64);
+      int w = 0, wu = 0, s = 0, su = 0, pk = 0;
       for (int kg = 0; kg < KT && ok; ++kg) {
-        const int w = kg % WS;
-        ok = mbar_wait_cluster(&ctl->wfull[w], static_cast<uint32_t>((kg / WS) & 1), deadline, abort_flag);
+        ok = mbar_wait_cluster(&ctl->wfull[w], static_cast<uint32_t>(wu & 1), deadline, abort_flag);
         if (!ok) break;
         if (kg + WS < KT) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);   // the slot's next use
-        const int s = kg % XS;
-        ok = mbar_wait(&xfull[s], static_cast<uint32_t>((kg / XS) & 1), deadline, abort_flag);
+        ok = mbar_wait(&xfull[s], static_cast<uint32_t>(su & 1), deadline, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t waddr = smem_u32(smem + L.w_off + w * kWTile);
-        const uint32_t xaddr = smem_u32(smem + L.x_off + s * L.x_stride);
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint64_t adesc = smem_desc_noswizzle(waddr + kk * 2 * 2048, 2048, 128);
-          // x: NT rows of 64 bytes (64-byte swizzle), K-step kk = bytes 32 kk of each row
-          const uint64_t bdesc = smem_desc_sw64(xaddr + kk * 32, 8 * 64);
-          mma_f16_ss(tmem, adesc, bdesc, idesc_g, (kg > 0 || kk > 0) ? 1u : 0u);
-        }
+        // descriptor start addresses count 16-byte units: W slot w at w * kWTile, K-step kk
+        // of the W tile 4096 bytes on; x stage s at s * x_stride, K-step kk 32 bytes on
+        const uint64_t adesc = adesc0 + static_cast<uint64_t>((w * kWTile) >> 4);
+        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((s * L.x_stride) >> 4);
+        mma_f16_ss(tmem, adesc, bdesc, idesc_g, kg > 0 ? 1u : 0u);
+        mma_f16_ss(tmem, adesc + (4096 >> 4), bdesc + (32 >> 4), idesc_g, 1u);
         issued_any = true;
         tc_commit(&xempty[s]);
         if (kg + WS < KT) {
-          if (CN > 1) tc_commit_multicast(&ctl->wempty[w], static_cast<uint16_t>(1u << (kg % CN)));
+          if (CN > 1) tc_commit_multicast(&ctl->wempty[w], static_cast<uint16_t>(1u << pk));
           else tc_commit(&ctl->wempty[w]);
         }
+        if (++w == WS) { w = 0; ++wu; }
+        if (++s == XS) { s = 0; ++su; }
+        if (++pk == CN) pk = 0;
       }
       if (ok) {
         tc_commit(&ctl->accfull);
