@@ -429,14 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // of the cluster, each copy completing the receiver's barrier, and completes its own
       if (bar_any(1, kRb, failed)) {
         failed = true;
-      } else if (threadIdx.x == 0) {
+      } else if (threadIdx.x < CN) {
+        // lane c of warp 0 serves rank c, the copies issued in parallel
+        const int c = threadIdx.x;
         const uint8_t* src = smem + L.w_off + w * kWTile;
-        for (int c = 0; c < CN; ++c) {
-          if (c == rank) continue;
+        if (c == rank) {
+          mbar_complete_tx(&ctl->wfull[w], kWTile);
+        } else {
           bulk_s2cluster(mapa_shared(smem_u32(src), static_cast<uint32_t>(c)), src, kWTile,
                          mapa_shared(smem_u32(&ctl->wfull[w]), static_cast<uint32_t>(c)));
         }
-        mbar_complete_tx(&ctl->wfull[w], kWTile);
       }
     }
     // epilogue: accumulator row `tid` holds NT token outputs; the two halves take
