@@ -700,22 +700,36 @@ def main():
     t_roof = max(nbytes / (hbm * 1e9), res["flops_factored"] / (bf16 * 1e12))
     traffic = dram_traffic("decode")
     cpu = run_oracle(args, budget_s=args.cpu_seconds) if args.cpu_seconds > 0 else None
+    if kind == "decode":
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic, "peak_source": src,
+                "t_roof_us": round(t_roof * 1e6, 3), "frac_of_roofline_time": round(t_roof * 1e6 / us_step, 4),
+                "bytes_per_launch": nbytes,
+                "tensor_i8_frac": round(2 * res["flops_factored"] * 1.0 / (us_step * 1e-6) / (i8_peak * 1e12), 4)}
+    else:
+        # the prefill kernel is a dense fp16/bf16 contraction: its roofline is the tensor
+        # peak, counted on the product's 2 batch m d FLOPs alone (the rank-k rebuild's
+        # 2 m d k n are extra work the kernel also does); the burst peak, the lower
+        # fraction of the two
+        gemm_flops = 2.0 * args.batch * args.m * args.d
+        tflops = gemm_flops / (us_step * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": bf16, "unit": "TFLOP/s",
+                "frac": round(tflops / bf16, 4), "traffic": dram_traffic("prefill"), "peak_source": src,
+                "flops_per_launch": gemm_flops, "rebuild_flops_per_launch": res["flops_rebuild"] - gemm_flops,
+                "bytes_per_launch": nbytes}
     line = {
-        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if args.batch == B_HEAD else METRIC.replace(f"batch {B_HEAD}", f"batch {args.batch}"),
+        "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us_step / 1000.0, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "vs_baseline": None, "dtype": "i8" if kind == "decode" else "f16", "data": "synthetic",
         "config": dict(config, l2_policy=f"inputs larger than L2: {res['n_stacks']} distinct stacks "
                                          f"({res['n_stacks'] * nbytes / 2**20:.0f} MiB) rotated, L2 "
                                          f"{res['l2'] / 2**20:.0f} MiB", timing="CUDA graph replays, CUDA events"),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": traffic, "peak_source": src,
-                     "t_roof_us": round(t_roof * 1e6, 3), "frac_of_roofline_time": round(t_roof * 1e6 / us_step, 4),
-                     "bytes_per_launch": nbytes,
-                     "tensor_i8_frac": round(2 * res["flops_factored"] * 1.0 / (us_step * 1e-6) / (i8_peak * 1e12), 4)},
+        "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": round(job_us_per_call(res["ms_e2e"], res["e2e_steps"], world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": res["e2e_h2d"], "d2h_bytes_per_step": res["e2e_d2h"]},
-        "gpu_launches": args.steps,       # one decode kernel per call
+        "gpu_launches": args.steps,       # one kernel (decode or prefill) per call
         "clocks": res["clocks"],
         "tokens_per_s": round(args.batch * 1e6 / value, 1),
         "weights_per_s": round(args.m * args.d * 1e6 / value, 1),
