@@ -100,11 +100,17 @@ size_t bs_block_bytes(int m, int d, int k);
 size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks);
 
 /* Workspace bytes bs_linear needs for `n_loaded` blocks and `batch` rows (0 when the
- * call needs none, i.e. n_loaded == 0 or batch > 4): one arrival counter per 128-row
- * tile (first, so its place never moves), then one fp32 partial output per (128-row
- * tile, chunk group of 4 x 256 columns at batch 1, else 2 x 256) and batch row, about
- * m * d * n * batch / 256 bytes at batch 1 and m * d * n * batch / 128 above.  The
- * caller zeroes a workspace once before its first use (e.g. cudaMemsetAsync); every
+ * call needs none).  Decode (batch <= 4): one arrival counter per 128-row tile (first,
+ * so its place never moves), then one fp32 partial output per (128-row tile, chunk
+ * group of 4 x 256 columns at batch 1, else 2 x 256) and batch row, about
+ * m * d * n * batch / 256 bytes at batch 1 and m * d * n * batch / 128 above.
+ * Prefill (batch > 4): none when its grid (128-row tiles x token tiles) fills the
+ * current device's SMs; otherwise the kernel splits K into s parts of whole 256-column
+ * groups, as many as fit beside the grid in one wave, and needs one counter per
+ * (row tile, token tile), 256-aligned, then s fp32 partial tiles of 128 rows x the
+ * token tile each (e.g. 16 tokens of a 4096 x 14336 weight on 148 SMs: s = 4, 2 MiB).
+ * A prefill call given a smaller workspace (or none) runs one pass over K instead.
+ * The caller zeroes a workspace once before its first use (e.g. cudaMemsetAsync); every
  * call that completes leaves its counters at zero again, so no clearing is needed
  * between calls, and calls captured in a CUDA graph may be replayed.  After a call
  * that reported BS_ERR_TIMEOUT the counters may be left non-zero: zero the workspace
@@ -167,11 +173,12 @@ bs_status bs_drop_block(bs_stack_t stack);
  * BS_BF16), device pointers, 16-byte aligned.  n_loaded == 0 writes y = 0 (the
  * restoration accumulator starts at zero).  batch <= 4 runs the decode path (the
  * factored form y = sum_i U_i (S_i ((x (.) 1/s) V_i)) with the +-1 contraction on
- * int8 tensor cores: a small kernel quantises the activations once per call, then
- * the contraction kernel); larger batches run the prefill kernel (W_hat tiles rebuilt
- * in shared memory, then a tcgen05 GEMM).  workspace: >= bs_workspace_bytes(m, d, k,
- * n_loaded, batch) device bytes, 256-aligned, zeroed before its first use (may be
- * NULL when the size is 0).  Asynchronous on `stream`; capturable in a CUDA graph.
+ * int8 tensor cores, in one kernel that also quantises the activations); larger
+ * batches run the prefill kernel (W_hat tiles rebuilt in shared memory, then a
+ * tcgen05 GEMM; K split across CTAs when the grid would leave SMs idle and the
+ * workspace holds the partials).  workspace: >= bs_workspace_bytes(m, d, k, n_loaded,
+ * batch) device bytes, 256-aligned, zeroed before its first use (may be NULL when the
+ * size is 0).  Asynchronous on `stream`; capturable in a CUDA graph.
  * The decode kernels are launched with programmatic dependent launch: they may start,
  * and read the stack's block area and the scale vector, before the kernel ahead of
  * them on `stream` has finished; they read x and touch the workspace and y only after

@@ -1,6 +1,7 @@
 // Host implementation of the C ABI declared in include/bitstack.h: argument checks,
 // the stack handle, block append/drop, host packing, and kernel dispatch.  The
 // library never allocates device memory; every device buffer comes from the caller.
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -111,6 +112,49 @@ GroupWs group_ws(int n_linears, const bs_stack_t* stacks, const int* n_loaded, i
 
 }  // namespace
 
+// Token tile: 256 for long inputs, 128 up to 2047 tokens (more CTAs to fill the SMs),
+// else the input rounded up to 32.  The CTAs of a row tile are clustered by up to 4 along
+// the tokens to share the rebuild of W_hat.  Shared memory: fewer x stages first (down to
+// two), then one sign buffer, then smaller token tiles, then a smaller cluster.  A grid
+// that would leave SMs idle splits K into as many parts (of whole sign groups) as fit
+// beside it in one wave.
+bool bs::prefill_config(int m, int d, int n, int batch, int sms, PrefillConfig* c) {
+  const size_t limit = 227 * 1024;
+  const int NT0 = batch >= 2048 ? 256 : (batch >= 128 ? 128 : ((batch + 31) / 32) * 32);
+  const int tiles0 = (batch + NT0 - 1) / NT0;
+  int CN = tiles0 >= 4 ? 4 : (tiles0 >= 2 ? 2 : 1);
+  int NT = NT0, xs = 4, sb = 2;
+  for (;;) {
+    xs = 4;
+    sb = 2;
+    NT = NT0;
+    while (prefill_smem_bytes(n, NT, xs, sb, CN) > limit && xs > 2) --xs;
+    if (prefill_smem_bytes(n, NT, xs, sb, CN) > limit) sb = 1;
+    while (prefill_smem_bytes(n, NT, xs, sb, CN) > limit && NT > 32) NT /= 2;
+    if (prefill_smem_bytes(n, NT, xs, sb, CN) <= limit) break;
+    if (CN == 1) return false;
+    CN /= 2;
+  }
+  c->NT = NT;
+  c->CN = CN;
+  c->xstages = xs;
+  c->sbufs = sb;
+  c->tiles = (batch + NT - 1) / NT;
+  c->gy = (c->tiles + CN - 1) / CN * CN;
+  const int KT = d / 32;   // 32-column K-tiles (a multiple of 8: d is a multiple of 256)
+  const long long ctas = static_cast<long long>(m / kTileRows) * c->gy;
+  int ks = 1;
+  if (sms > 0 && ctas < sms) ks = std::min(static_cast<int>(sms / ctas), (KT + 7) / 8);
+  int kts = ((KT + ks - 1) / ks + 7) / 8 * 8;
+  ks = (KT + kts - 1) / kts;
+  c->ks = ks;
+  c->kts = kts;
+  const size_t tiles_all = static_cast<size_t>(m / kTileRows) * c->tiles;
+  c->cnt_bytes = ks > 1 ? (tiles_all * 4 + 255) / 256 * 256 : 0;
+  c->part_bytes = ks > 1 ? static_cast<size_t>(ks) * tiles_all * kTileRows * NT * 4 : 0;
+  return true;
+}
+
 extern "C" {
 
 size_t bs_block_bytes(int m, int d, int k) {
@@ -125,8 +169,17 @@ size_t bs_stack_device_bytes(int m, int d, int k, int capacity_blocks) {
 
 size_t bs_workspace_bytes(int m, int d, int k, int n_loaded, int batch) {
   if (!gpu_shape_ok(m, d, k) || n_loaded < 0 || batch <= 0) return 0;
-  if (n_loaded == 0 || batch > kDecodeMaxBatch) return 0;
-  return decode_ws_layout(m, d, n_loaded, batch).total;
+  if (n_loaded == 0) return 0;
+  if (batch <= kDecodeMaxBatch) return decode_ws_layout(m, d, n_loaded, batch).total;
+  // the prefill's split-K partials, for the current device's SM count (148 without one)
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  PrefillConfig cfg;
+  if (!prefill_config(m, d, n_loaded, batch, sms, &cfg)) return 0;
+  return cfg.cnt_bytes + cfg.part_bytes;
 }
 
 bs_status bs_pack_record(int m, int d, int k, const uint8_t* neg_bits, const uint16_t* U, const uint16_t* V,
@@ -361,31 +414,25 @@ bs_status bs_linear(bs_stack_t stack, const void* x, int batch, bs_dtype dt, int
   p.n = n_loaded;
   p.M = batch;
   p.KG = d / kTileCols;
-  // Token tile: 256 for long inputs, 128 up to 2047 tokens (more CTAs to fill the SMs),
-  // else the input rounded up to 32.  The CTAs of a row tile are clustered by up to 4
-  // along the tokens to share the rebuild of W_hat.
-  p.NT = batch >= 2048 ? 256 : (batch >= 128 ? 128 : ((batch + 31) / 32) * 32);
-  const int tiles = (batch + p.NT - 1) / p.NT;
-  p.CN = tiles >= 4 ? 4 : (tiles >= 2 ? 2 : 1);
   p.timeout_ns = stack->timeout_ns;
-  // Shared memory: fewer x stages first (down to two), then one sign buffer, then smaller
-  // token tiles, then a smaller cluster.
-  const size_t limit = 227 * 1024;
-  const int NT0 = p.NT;
-  int xs = 4, sb = 2;
-  for (;;) {
-    xs = 4;
-    sb = 2;
-    p.NT = NT0;
-    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && xs > 2) --xs;
-    if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit) sb = 1;
-    while (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) > limit && p.NT > 32) p.NT /= 2;
-    if (prefill_smem_bytes(n_loaded, p.NT, xs, sb, p.CN) <= limit) break;
-    if (p.CN == 1) return BS_ERR_CAPACITY;
-    p.CN /= 2;
+  PrefillConfig cfg;
+  if (!prefill_config(m, d, n_loaded, batch, stack->sm_count, &cfg)) return BS_ERR_CAPACITY;
+  p.NT = cfg.NT;
+  p.CN = cfg.CN;
+  p.xstages = cfg.xstages;
+  p.sbufs = cfg.sbufs;
+  p.tiles_y = cfg.tiles;
+  p.ks = 1;
+  p.kts = d / 32;           // one split: all 32-column K-tiles
+  // split K only with a workspace that holds the partials (else one pass over K)
+  if (cfg.ks > 1 && workspace != nullptr && workspace_bytes >= cfg.cnt_bytes + cfg.part_bytes) {
+    if (!aligned(workspace, 256)) return BS_ERR_ALIGNMENT;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.ks = cfg.ks;
+    p.kts = cfg.kts;
+    p.cnt = reinterpret_cast<uint32_t*>(ws);
+    p.part = reinterpret_cast<float*>(ws + cfg.cnt_bytes);
   }
-  p.xstages = xs;
-  p.sbufs = sb;
   CUtensorMap tm_x;
   const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(batch)};
   const cuuint64_t xstr[1] = {static_cast<cuuint64_t>(d) * 2};

@@ -90,7 +90,23 @@ struct PrefillParams {
   int xstages, sbufs;
   int CN;                      // CTAs per cluster along the tokens sharing the W_hat rebuild (1, 2, 4)
   unsigned long long timeout_ns;
+  // Split K (grids that would leave SMs idle): split z takes the K-tiles [z kts, (z + 1) kts)
+  // (kts a multiple of 8, the K-tiles of one sign group) and writes an fp32 partial tile;
+  // the CTA that counts a tile's last partial sums the ks partials in split order into y.
+  int ks, kts, tiles_y;        // splits, K-tiles per split, token tiles that hold tokens
+  float* part;                 // [row tile][token tile][split][128 x NT] partial tiles
+  uint32_t* cnt;               // [row tile][token tile] arrival counters, zero between calls
 };
+
+// Launch shape of the prefill kernel for a call (host side; also sizes its workspace).
+struct PrefillConfig {
+  int NT, CN, xstages, sbufs;  // token tile, cluster size, x stages, sign buffers
+  int ks, kts;                 // K splits and K-tiles per split
+  int tiles, gy;               // token tiles holding tokens, and padded to whole clusters
+  size_t cnt_bytes, part_bytes;  // workspace: counters (256-aligned), then partials
+};
+// False when no configuration fits in shared memory (n too large).
+bool prefill_config(int m, int d, int n, int batch, int sms, PrefillConfig* cfg);
 
 // "w/o AVD" stacks: blocks that are plain rank-k' factor pairs, record = [U m x k' fp16
 // row-major][V d x k' fp16 row-major].  k' is a multiple of 8 (whole 16-byte rows), at

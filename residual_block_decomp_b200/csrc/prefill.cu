@@ -59,6 +59,7 @@ struct Ctl {
   uint64_t vfull[kVS], vempty[kVS];  // V stages of the own K-tiles
   uint32_t tmem_base;
   int abort;
+  int last;                          // split K: this CTA counted its tile's last partial
 };
 
 template <typename DT>
@@ -121,8 +122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rt = blockIdx.x;
   const int tok0 = blockIdx.y * NT;
   const int rank = CN > 1 ? static_cast<int>(cluster_rank()) : 0;
-  const int KT = p.d / kKT;
-  const int n_own = (KT - rank + CN - 1) / CN;      // own K-tiles rank, rank + CN, ...
+  // this split's K-tiles kt0 .. kt0 + KT - 1 (kt0 a multiple of 8: whole sign groups);
+  // below, kl = kt - kt0 indexes them
+  const int kt0 = static_cast<int>(blockIdx.z) * p.kts;
+  const int KT = min(p.kts, p.d / kKT - kt0);
+  const int n_own = (KT - rank + CN - 1) / CN;      // own K-tiles kl = rank, rank + CN, ...
   const int rounds = (n + kPRound - 1) / kPRound;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
   const uint32_t is_bf16 = std::is_same<DT, __nv_bfloat16>::value ? 1u : 0u;
@@ -170,16 +174,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t FULL = 0xffffffffu;
     if (lane == 0) prefetch_tmap(&tm_x);
     bool ok = true;
-    int kt = 0;
-    for (; kt < KT && ok; ++kt) {
-      const int s = kt % XS, use = kt / XS;
+    int kl = 0;
+    for (; kl < KT && ok; ++kl) {
+      const int s = kl % XS, use = kl / XS;
       if (lane == 0) {
         if (use > 0) ok = mbar_wait(&xempty[s], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
         if (ok) mbar_arrive_expect_tx(&xfull[s], static_cast<uint32_t>(NT) * kKT * 2u);
       }
       ok = __shfl_sync(FULL, ok, 0);
       if (!ok) break;
-      if (lane == 0) tma_load_2d(smem + L.x_off + s * L.x_stride, &tm_x, kt * kKT, tok0, &xfull[s]);
+      if (lane == 0) tma_load_2d(smem + L.x_off + s * L.x_stride, &tm_x, (kt0 + kl) * kKT, tok0, &xfull[s]);
     }
     if (lane == 0) {
       if (!ok) {
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(p.err, kErrTimeout);
       }
       const uint64_t drain_by = globaltimer_ns() + 100000000ull;
-      for (int j = (kt > XS ? kt - XS : 0); j < kt; ++j)
+      for (int j = (kl > XS ? kl - XS : 0); j < kl; ++j)
         mbar_wait(&xfull[j % XS], static_cast<uint32_t>((j / XS) & 1), drain_by, nullptr);
     }
   } else if (warp == kWarpRbLoad) {
@@ -208,9 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int oi = 0, groups = 0;
     for (; oi < n_own && ok; ++oi) {
-      const int kt = rank + oi * CN;
-      if (oi == 0 || (kt - CN) / 8 != kt / 8) {   // the first own K-tile of a sign group
-        const int grp = kt / 8, sb = grp % SB, use = grp / SB;
+      const int kl = rank + oi * CN, kt = kt0 + kl;
+      if (oi == 0 || (kl - CN) / 8 != kl / 8) {   // the first own K-tile of a sign group
+        // buffers and phases count the split's groups; the source is the global group
+        const int grp = kt / 8, lg = kl / 8, sb = lg % SB, use = lg / SB;
         if (lane == 0) {
           if (use > 0) ok = mbar_wait(&sgempty[sb], static_cast<uint32_t>((use - 1) & 1), deadline, abort_flag);
           if (ok) mbar_arrive_expect_tx(&sgfull[sb], static_cast<uint32_t>(n) * kTileBytes);
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool issued_any = false;
       // every W slot expects one tile's bytes for its first use
-      for (int w = 0; w < WS && w < KT; ++w) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);
+      for (int w = 0; w < WS && w < KT; ++w) mbar_arrive_expect_tx(&ctl->wfull[w], kWTile);   // split-local
       // ring positions kept as counters (no divisions in the loop): W slot w of use wu,
       // x stage s of use su, producer rank pk = kg mod CN
       const uint64_t adesc0 = smem_desc_noswizzle(smem_u32(smem + L.w_off), 2048, 128);
@@ -348,16 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) failed = true;
     };
     int prounds = 0;
-    // the CTA's own K-tiles kt = rank, rank + CN, ...; each is written into ring slot
-    // kt mod WS of every CTA of the cluster
+    // the CTA's own K-tiles kl = rank, rank + CN, ... of the split; each is written into
+    // ring slot kl mod WS of every CTA of the cluster
     for (int oi = 0; oi < n_own; ++oi) {
-      const int kt = rank + oi * CN;
-      const int grp = kt / 8, t = kt % 8, sb = grp % SB;
-      const int w = kt % WS;
-      const bool first_in_group = oi == 0 || (kt - CN) / 8 != grp;
-      const bool last_in_group = oi + 1 == n_own || (kt + CN) / 8 != grp;
+      const int kl = rank + oi * CN, kt = kt0 + kl;
+      const int lg = kl / 8, t = kl % 8, sb = lg % SB;   // the split's group, K-tile in it
+      const int w = kl % WS;
+      const bool first_in_group = oi == 0 || (kl - CN) / 8 != lg;
+      const bool last_in_group = oi + 1 == n_own || (kl + CN) / 8 != lg;
       if (first_in_group && !failed)
-        check(mbar_wait(&sgfull[sb], static_cast<uint32_t>((grp / SB) & 1), deadline, abort_flag));
+        check(mbar_wait(&sgfull[sb], static_cast<uint32_t>((lg / SB) & 1), deadline, abort_flag));
       // column c of the K-tile is bit 8 (c % 4) + t of word c / 4 of the row; a multiply by
       // 2^(31 - 8 (c % 4) - t) moves it to bit 31 on the FMA pipe, leaving one AND-XOR
       // (the integer pipe) and one add per element and block
@@ -413,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 16; c += 2) packed[c / 2] = pack2<DT>(acc[c] * isv[c], acc[c + 1] * isv[c + 1]);
       // the slot is free in every CTA of the cluster once all their GEMMs of the tile
       // WS earlier (also this rank's) are done
-      if (kt >= WS && !failed)
-        check(mbar_wait_cluster(&ctl->wempty[w], static_cast<uint32_t>(((kt / WS) - 1) & 1), deadline, abort_flag));
+      if (kl >= WS && !failed)
+        check(mbar_wait_cluster(&ctl->wempty[w], static_cast<uint32_t>(((kl / WS) - 1) & 1), deadline, abort_flag));
       if (!failed) {
 #pragma unroll
         for (int k2 = 0; k2 < 2; ++k2) {
@@ -442,23 +447,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // epilogue: accumulator row `tid` holds NT token outputs; the two halves take
-    // alternate 32-column chunks
+    // alternate 32-column chunks.  Without a K split they go to y; with one, to this
+    // split's fp32 partial tile (token-major, rows contiguous).  The CTAs that pad the
+    // token tiles to whole clusters store nothing.
     if (!failed) check(mbar_wait(&ctl->accfull, 0, deadline, abort_flag));
-    if (!failed) {
+    const bool real = tok0 < p.M;
+    DT* y = static_cast<DT*>(p.y);
+    const size_t row = static_cast<size_t>(rt) * kTileRows + tid;
+    const size_t tile = static_cast<size_t>(rt) * p.tiles_y + blockIdx.y;
+    if (!failed && real) {
       tc_fence_after();
-      DT* y = static_cast<DT*>(p.y);
-      const size_t row = static_cast<size_t>(rt) * kTileRows + tid;
+      float* part = p.ks > 1 ? p.part + (tile * p.ks + blockIdx.z) * (kTileRows * NT) : nullptr;
       for (int ch = half; ch < NT / 32; ch += 2) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + ch * 32, v);
         tc_wait_ld();
+        if (part != nullptr) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tok = tok0 + ch * 32 + j;
-          if (tok < p.M) y[static_cast<size_t>(tok) * p.m + row] = cvt_out<DT>(__uint_as_float(v[j]));
+          for (int j = 0; j < 32; ++j) part[(ch * 32 + j) * kTileRows + tid] = __uint_as_float(v[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = tok0 + ch * 32 + j;
+            if (tok < p.M) y[static_cast<size_t>(tok) * p.m + row] = cvt_out<DT>(__uint_as_float(v[j]));
+          }
         }
       }
       tc_fence_before();
+    }
+    if (p.ks > 1 && real) {
+      // count this partial; the CTA that adds the tile's last one sums all of them in
+      // split order (the same association whichever CTA it is) and writes y.  No CTA
+      // waits for another.  A CTA that failed counts nothing: its tile is never written
+      // and the error word tells the caller (who zeroes the workspace again).
+      __threadfence();
+      if (bar_any(1, kRb, failed)) {
+        failed = true;
+      } else {
+        if (threadIdx.x == 0)
+          ctl->last = atomicAdd(p.cnt + tile, 1u) == static_cast<uint32_t>(p.ks - 1) ? 1 : 0;
+        bar_named(1, kRb);
+        if (ctl->last) {
+          __threadfence();
+          const float* part = p.part + tile * p.ks * (kTileRows * NT);
+          for (int ch = half; ch < NT / 32; ch += 2) {
+            for (int j = 0; j < 32; ++j) {
+              const int tl = ch * 32 + j;
+              if (tok0 + tl >= p.M) break;
+              float acc = 0.0f;
+              for (int z = 0; z < p.ks; ++z) acc += __ldcg(part + (static_cast<size_t>(z) * NT + tl) * kTileRows + tid);
+              y[static_cast<size_t>(tok0 + tl) * p.m + row] = cvt_out<DT>(acc);
+            }
+          }
+          if (threadIdx.x == 0) p.cnt[tile] = 0u;   // left at zero for the next call
+        }
+      }
     }
     if (failed) {
       ctl->abort = 1;
@@ -513,7 +556,7 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tm_x, cons
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.stream = stream;
-  cfg.gridDim = dim3(static_cast<unsigned>(p.m / kTileRows), static_cast<unsigned>(gy));
+  cfg.gridDim = dim3(static_cast<unsigned>(p.m / kTileRows), static_cast<unsigned>(gy), static_cast<unsigned>(p.ks));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   if (bf16) return cudaLaunchKernelEx(&cfg, prefill_kernel<__nv_bfloat16>, p, tm_x, tm_u, tm_v);

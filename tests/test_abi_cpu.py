@@ -53,7 +53,13 @@ def test_device_and_workspace_sizes():
     assert ws == 32 * (16 // 4) * 8 * 128 * 4 + 256
     assert R.bs_workspace_bytes(4096, 4096, 16, 8, 4) > ws
     assert R.bs_workspace_bytes(4096, 4096, 16, 0, 1) == 0    # n = 0 needs none
-    assert R.bs_workspace_bytes(4096, 4096, 16, 8, 64) == 0   # prefill needs none
+    # prefill: a grid that fills the SMs needs none; 64 tokens (32 CTAs) split K in 4
+    # (148 SMs assumed without a device): 256 bytes of counters, then 4 partial tiles
+    # of 128 rows x 64 tokens per row tile
+    assert R.bs_workspace_bytes(4096, 4096, 16, 8, 4096) == 0
+    assert R.bs_workspace_bytes(4096, 4096, 16, 8, 64) == 256 + 4 * 32 * 128 * 64 * 4
+    # 16 tokens of the 4096 x 14336 MLP weight: 4 splits of 112 K-tiles, 32-token tiles
+    assert R.bs_workspace_bytes(4096, 14336, 16, 8, 16) == 256 + 4 * 32 * 128 * 32 * 4
 
 
 @pytest.mark.parametrize("m,d,seed", [(128, 256, 0), (256, 512, 1), (384, 768, 2), (512, 512, 3)])
