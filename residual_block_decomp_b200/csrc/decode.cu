@@ -43,8 +43,10 @@
 //    batch row; they zero the accumulator for reuse (every MMA accumulates; int32 sums
 //    are exact, so the order of the units does not matter).
 //  * Reduction.  At the end every CTA counts its partials into per-row-tile arrival
-//    counters; the CTA that adds a tile's last partial sums all of them in fixed
-//    chunk-group order and writes y: deterministic, and no CTA ever waits for another.
+//    counters (acquire-release atomics at GPU scope, which publish the partials and
+//    make the others' visible to the last arrival); the CTA that adds a tile's last
+//    partial sums all of them in fixed chunk-group order and writes y: deterministic,
+//    and no CTA ever waits for another.
 //  * Hand-overs between roles are mbarriers, waited on with the suspending try_wait so
 //    that a waiting warp takes no issue slots from the warps that expand signs.
 //  * Every wait is bounded; a wait that runs out sets the device error word, and the
@@ -833,7 +835,6 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const __grid
           ++zk;
         }
       }
-      __threadfence();   // this thread's partials are visible before any arrival is counted
       const bool stop = bar_any(kBarEpi, 128, failed || *abort_flag != 0);
       if (et == 0) ctl->count_ok = stop ? 0 : 1;
     }
@@ -860,14 +861,16 @@ __global__ void __launch_bounds__(Cfg<B>::THREADS, 1) decode_kernel(const __grid
       if (e < nseg) {
         const Seg se = seg_of(s0 + e, p, C);
         const DecodeLin& L = lin_at(p, se.l);
-        if (atomicAdd(L.cnt + se.rt, 1u) == static_cast<uint32_t>(L.n * L.NCB - 1)) {
+        // acquire-release at GPU scope: releases this CTA's partials (the barrier above
+        // orders every thread's stores before it) and, for the last arrival, acquires
+        // all the others' (the barrier below orders this CTA's reads after it)
+        if (atom_add_acq_rel_gpu(L.cnt + se.rt, 1u) == static_cast<uint32_t>(L.n * L.NCB - 1)) {
           const int idx = atomicAdd(&ctl->nred, 1);
           red_rt[idx] = (se.l << 16) | se.rt;
         }
       }
       __syncthreads();
       const int nred = ctl->nred;
-      if (nred > 0) __threadfence();
       // up to kTB row tiles per pass, their loads all in flight together
       constexpr int kTB = 4;
       for (int q0 = 0; q0 < nred; q0 += kTB) {

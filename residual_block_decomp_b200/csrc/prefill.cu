@@ -479,16 +479,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // count this partial; the CTA that adds the tile's last one sums all of them in
       // split order (the same association whichever CTA it is) and writes y.  No CTA
       // waits for another.  A CTA that failed counts nothing: its tile is never written
-      // and the error word tells the caller (who zeroes the workspace again).
-      __threadfence();
+      // and the error word tells the caller (who zeroes the workspace again).  The count
+      // is an acquire-release atomic at GPU scope: after the barrier it releases every
+      // rebuild thread's partial stores, and for the last arrival it acquires the other
+      // CTAs' (the barrier after it orders this CTA's reads behind it).
       if (bar_any(1, kRb, failed)) {
         failed = true;
       } else {
         if (threadIdx.x == 0)
-          ctl->last = atomicAdd(p.cnt + tile, 1u) == static_cast<uint32_t>(p.ks - 1) ? 1 : 0;
+          ctl->last = atom_add_acq_rel_gpu(p.cnt + tile, 1u) == static_cast<uint32_t>(p.ks - 1) ? 1 : 0;
         bar_named(1, kRb);
         if (ctl->last) {
-          __threadfence();
           const float* part = p.part + tile * p.ks * (kTileRows * NT);
           for (int ch = half; ch < NT / 32; ch += 2) {
             for (int j = 0; j < 32; ++j) {

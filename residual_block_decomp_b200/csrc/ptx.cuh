@@ -165,6 +165,12 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------- global flags -------
+// atomic add with acquire-release semantics at GPU scope; returns the old value
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
