@@ -60,6 +60,16 @@ def test_device_and_workspace_sizes():
     assert R.bs_workspace_bytes(4096, 4096, 16, 8, 64) == 256 + 4 * 32 * 128 * 64 * 4
     # 16 tokens of the 4096 x 14336 MLP weight: 4 splits of 112 K-tiles, 32-token tiles
     assert R.bs_workspace_bytes(4096, 14336, 16, 8, 16) == 256 + 4 * 32 * 128 * 32 * 4
+    # 14336 rows: 112 CTAs already fill the SMs' one wave (148 // 112 = 1 split): none
+    assert R.bs_workspace_bytes(14336, 4096, 16, 8, 16) == 0
+    # one row tile, 600 tokens of 2560 columns: 5 token tiles of 128 in clusters of 4
+    # (8 CTAs with the padding) -> min(148 // 8, 80 // 8) = 10 splits of 8 K-tiles;
+    # counters for 1 x 5 tiles, then 10 partial tiles of 128 x 128 per token tile
+    assert R.bs_workspace_bytes(128, 2560, 16, 5, 600) == 256 + 10 * 5 * 128 * 128 * 4
+    # 16 loaded blocks fit the prefill's shared memory at 64 tokens; 40 do not (U, V and
+    # one sign group alone pass 227 KB)
+    assert R.bs_workspace_bytes(128, 4096, 16, 16, 64) > 0
+    assert R.bs_workspace_bytes(128, 4096, 16, 40, 64) == 0
 
 
 @pytest.mark.parametrize("m,d,seed", [(128, 256, 0), (256, 512, 1), (384, 768, 2), (512, 512, 3)])
