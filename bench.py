@@ -253,23 +253,47 @@ def run_cuda(args, rank, world, local_rank):
         assert layer.device_error() == 0, "device error in the timed region"
 
     # ------------------------------------------------------------------ e2e ----
-    # through the C ABI with host buffers: pinned x -> device, bs_linear, y -> pinned host
+    # through the C ABI with host buffers: every call copies its x from pinned host memory,
+    # runs bs_linear and copies its y back to pinned host memory.  As a serving loop would,
+    # the copies run on their own streams and overlap the neighbouring calls' kernels: call
+    # j's kernel waits for its x, its y copy waits for its kernel, and a buffer is reused
+    # (x refilled, y overwritten) only after its previous call has consumed it.
     xh = [torch.empty((b, d), dtype=torch.float16, pin_memory=True) for _ in range(n_stacks)]
     yh = [torch.empty((b, m), dtype=torch.float16, pin_memory=True) for _ in range(n_stacks)]
     for j in range(n_stacks):
         xh[j].copy_(xs[j].cpu())
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(n_stacks)]     # x of buffer jj landed
+    ev_done = [torch.cuda.Event() for _ in range(n_stacks)]   # its call finished (x read, y written)
+    ev_out = [torch.cuda.Event() for _ in range(n_stacks)]    # its y copied out
 
     def e2e_step(j):
         jj = j % n_stacks
-        xs[jj].copy_(xh[jj], non_blocking=True)
+        with torch.cuda.stream(h2d):
+            if j >= n_stacks:
+                h2d.wait_event(ev_done[jj])
+            xs[jj].copy_(xh[jj], non_blocking=True)
+            ev_in[jj].record(h2d)
+        stream.wait_event(ev_in[jj])
+        if j >= n_stacks:
+            stream.wait_event(ev_out[jj])
         step(jj)
-        yh[jj].copy_(ys[jj], non_blocking=True)
+        ev_done[jj].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_done[jj])
+            yh[jj].copy_(ys[jj], non_blocking=True)
+            ev_out[jj].record(d2h)
 
     def capture_e2e(count):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
+            h2d.wait_stream(stream)
+            d2h.wait_stream(stream)
             for j in range(count):
                 e2e_step(j)
+            stream.wait_stream(h2d)
+            stream.wait_stream(d2h)
         return g
 
     e2e_steps = args.e2e_steps or args.steps
